@@ -1,0 +1,78 @@
+"""KV-chunked attention and the exact log-sum-exp merge (test infrastructure).
+
+Ring attention streams K/V chunks past a rank's queries and keeps an online
+softmax, so no rank holds all of K/V (TensorRT 11.0 multi-device article,
+section on the three context-parallel implementations, Ring Attention).  On
+one device this is: split the keys into ``P`` contiguous chunks, compute a
+partial result per chunk, merge the partials.  For chunk ``p`` (keys
+``[floor(p*S/P), floor((p+1)*S/P))``) the partial is plain attention over
+those keys only:
+
+    o_p, lse_p = attention(q, k[chunk p], v[chunk p])
+
+and the merge (the split-reduction the accuracy table of "TensorRT
+Multi-Device (multi-GPU) support", Validation, attributes its FP16 error to):
+
+    L   = max_p lse_p
+    lse = L + ln(sum_p exp(lse_p - L))
+    o   = sum_p exp(lse_p - lse) * o_p
+
+which equals monolithic attention in exact arithmetic.  An empty chunk has
+``lse_p = -inf`` and ``o_p = 0`` and contributes nothing.  This module does
+not import ``oracle.attention``'s merge logic (there is none there); it calls
+``attention`` only to produce each chunk's partial.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .attention import attention
+
+
+def chunk_bounds(S: int, P: int):
+    """Contiguous chunk ``p`` covers keys ``[floor(p*S/P), floor((p+1)*S/P))``."""
+    return [((p * S) // P, ((p + 1) * S) // P) for p in range(P)]
+
+
+def partials(q, k, v, scale: float, P: int, rows=None):
+    """Per-chunk partials: ``o_parts [P, R, H, d]``, ``lse_parts [P, H, R]``."""
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    o_list, l_list = [], []
+    for lo, hi in chunk_bounds(k.shape[0], P):
+        o_p, lse_p = attention(q, k[lo:hi], v[lo:hi], scale, rows=rows)
+        o_list.append(o_p)
+        l_list.append(lse_p)
+    return np.stack(o_list), np.stack(l_list)
+
+
+def merge(o_parts, lse_parts):
+    """Exact merge of partials.
+
+    ``o_parts [P, S, H, d]`` and ``lse_parts [P, H, S]`` (any float dtype,
+    widened to float64) -> ``(o [S, H, d], lse [H, S])`` in float64.
+    Rows whose every chunk is empty get ``o = 0``, ``lse = -inf``.
+    """
+    o_parts = np.asarray(o_parts).astype(np.float64)
+    lse_parts = np.asarray(lse_parts).astype(np.float64)
+    P, S, H, d = o_parts.shape
+    L = lse_parts.max(axis=0)                                  # [H, S]
+    finite = np.isfinite(L)
+    L_safe = np.where(finite, L, 0.0)
+    w = np.exp(lse_parts - L_safe[None])                       # [P, H, S]
+    w = np.where(np.isneginf(lse_parts), 0.0, w)
+    total = w.sum(axis=0)                                      # [H, S]
+    lse = np.where(finite, L_safe + np.log(np.where(finite, total, 1.0)), -np.inf)
+    lse_safe = np.where(finite, lse, 0.0)
+    coef = np.exp(lse_parts - lse_safe[None])                  # exp(lse_p - lse)
+    coef = np.where(np.isneginf(lse_parts) | ~finite[None], 0.0, coef)
+    # o[s, h, :] = sum_p coef[p, h, s] * o_parts[p, s, h, :]
+    o = np.einsum("phs,pshd->shd", coef, o_parts)
+    return o, lse
+
+
+def chunked_attention(q, k, v, scale: float, P: int, rows=None):
+    """Partials over ``P`` chunks followed by the merge."""
+    o_parts, lse_parts = partials(q, k, v, scale, P, rows=rows)
+    return merge(o_parts, lse_parts)
