@@ -1,0 +1,412 @@
+"""Benchmark: non-causal long-sequence attention on B200, one JSON line.
+
+Default workload: S=32768, 32 heads x 128, Q ~ N(0, 4^2), K,V ~ N(0,1), fp16.
+One step = the whole hot path over that input: monolithic attention
+(attn_fwd) plus the ring-attention emulation (8 key-chunk partials with
+attn_fwd_partial, then attn_merge).  Both passes do 4*S^2*d*H flops, so the
+step's work is 2 * 4*S^2*d*H.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME]
+
+N > 1 runs under torchrun as N independent replicas (one per GPU, nothing
+exchanged on the data path); the timing is the max over ranks.  The
+``reference`` arm times the FP64 CPU oracle on a bounded sample of the same
+workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention TFLOP/s (4·S²·d·H, FP16) and % of B200 dense FP16 peak; ms/call"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.SEQ32K.name, choices=sorted(W.ATTN_WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------ distributed --
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- clocks --
+
+CLOCK_FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return False
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 9:
+                continue
+            self.rows.append(parts)
+        return False
+
+    def summary(self):
+        rows = getattr(self, "rows", [])
+        if self.bus_id:
+            mine = [r for r in rows if r[0].lower().endswith(self.bus_id.lower()[-12:])]
+            rows = mine or rows
+        buses = {r[0] for r in rows}
+        if len(buses) > 1:
+            rows = [r for r in rows if r[0] == sorted(buses)[0]]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "", 1).isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
+        reasons = sorted({name for r in rows for name, v in zip(REASONS, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def bus_id_of(device_index: int):
+    try:
+        import torch
+        p = torch.cuda.get_device_properties(device_index)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ peaks --
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": m["hbm_gbs"], "tc_burst": m["bf16_tflops"],
+                "tc_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]),
+                "source": "measured (MEASURED_PEAKS.json; fp16 dense rate = bf16 rate)"}
+    return {"hbm_gbs": 6650.0, "tc_burst": 1590.0, "tc_sustained": 1400.0,
+            "source": "fallback (profiling recipe figures)"}
+
+
+def committed_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    ent = table.get(kernel, {}).get(workload)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "long_context_bidirectional_b200", "csrc", ent["source"])
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != ent["source_sha256_16"]:
+            return None
+    return ent["bytes_per_launch"]
+
+
+# ---------------------------------------------------------- CPU baseline --
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_sample(w, rows_per_head: int):
+    """Time the FP64 oracle on ``rows_per_head`` query rows of every head."""
+    from oracle import attention as OA
+    q, k, v = W.workload_qkv(w)
+    rows = [W.sample_rows(w.S, 1, h, seed=w.seed, n=rows_per_head) for h in range(w.H)]
+    t0 = time.perf_counter()
+    OA.attention(q, k, v, w.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * rows_per_head * w.S * w.d * w.H
+    return flops, dt
+
+
+def cpu_baseline(w, budget_s: float = 10.0):
+    rows = 8
+    flops, dt = oracle_sample(w, rows)
+    while dt < budget_s / 4 and rows < 1024:
+        rows *= 2
+        flops, dt = oracle_sample(w, rows)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"FP64 numpy oracle, monolithic attention of {rows} query rows per head x "
+                      f"{w.H} heads against all {w.S} keys ({flops / 1e9:.1f} GFLOP in {dt:.2f} s); "
+                      f"host has {os.cpu_count()} logical cores"}
+
+
+# --------------------------------------------------------------- our arm --
+
+def run_ours(args, rank, world, local):
+    import torch
+    import long_context_bidirectional_b200 as b2a
+
+    w = W.ATTN_WORKLOADS[args.workload]
+    P = max(w.P, 1)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q, k, v = W.workload_qkv(w)
+    qd, kd, vd = (torch.from_numpy(x).to(dev) for x in (q, k, v))
+    S, H, d = w.S, w.H, w.d
+    out = torch.empty((S, H, d), dtype=torch.float16, device=dev)
+    lse = torch.empty((H, S), dtype=torch.float32, device=dev)
+    out_c = torch.empty_like(out)
+    lse_c = torch.empty_like(lse)
+    o_parts = torch.empty((P, S, H, d), dtype=torch.float32, device=dev)
+    lse_parts = torch.empty((P, H, S), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    bounds = b2a.chunk_bounds(S, P)
+
+    ev = {name: [] for name in ("mono", "partials", "merge")}
+
+    def step(record):
+        def mark():
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            return e
+        e0 = mark() if record else None
+        b2a.attn_fwd(qd, kd, vd, out=out, lse=lse, scale=w.scale, stream=stream)
+        e1 = mark() if record else None
+        for c, (lo, hi) in enumerate(bounds):
+            b2a.attn_fwd_partial(qd, kd[lo:hi], vd[lo:hi], o_parts[c], lse_parts[c], scale=w.scale,
+                                 stream=stream)
+        e2 = mark() if record else None
+        b2a.attn_merge(o_parts, lse_parts, out=out_c, lse_out=lse_c, stream=stream)
+        e3 = mark() if record else None
+        if record:
+            ev["mono"].append((e0, e1))
+            ev["partials"].append((e1, e2))
+            ev["merge"].append((e2, e3))
+
+    for _ in range(args.warmup):
+        step(False)
+    b2a.check_status(stream)
+    barrier(world)
+    torch.cuda.synchronize()
+
+    with ClockSampler(bus_id_of(local)) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    b2a.check_status(stream)
+    local_ms = t0.elapsed_time(t1) / args.steps
+    ms = reduce_max(local_ms, world)
+
+    def avg(name):
+        return sum(a.elapsed_time(b) for a, b in ev[name]) / len(ev[name])
+
+    mono_ms = reduce_max(avg("mono"), world)
+    part_ms = reduce_max(avg("partials"), world)
+    merge_ms = reduce_max(avg("merge"), world)
+
+    step_flops = 2.0 * w.flops
+    value = world * step_flops / (ms * 1e-3) / 1e12
+    pk = peaks()
+    mono_tflops = w.flops / (mono_ms * 1e-3) / 1e12
+    merge_bytes = P * S * H * d * 4 + P * H * S * 4 + S * H * d * 2 + H * S * 4
+    merge_gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
+
+    # end to end from pinned host memory through the C-ABI host entry point
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+        oh = torch.empty((S, H, d), dtype=torch.float16).pin_memory()
+        lh = torch.empty((H, S), dtype=torch.float32).pin_memory()
+        oh2 = torch.empty_like(oh).pin_memory()
+        lh2 = torch.empty_like(lh).pin_memory()
+        del o_parts, lse_parts
+        ws = torch.empty(b2a.host_workspace_bytes(S, H, d, P), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            b2a.attn_fwd_host(qh, kh, vh, oh, lh, ws, P=1, scale=w.scale, stream=stream)
+            b2a.attn_fwd_host(qh, kh, vh, oh2, lh2, ws, P=P, scale=w.scale, stream=stream)
+
+        for _ in range(max(1, min(args.warmup, 2))):
+            e2e_step()
+        b2a.check_status(stream)
+        barrier(world)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, world)
+        b2a.check_status(stream)
+        n16 = S * H * d * 2
+        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 2 * 3 * n16, "d2h_bytes_per_step": 2 * (n16 + H * S * 4),
+               "path": "attn_fwd_host(P=1) + attn_fwd_host(P=%d) from pinned host buffers" % P}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    clocks = clk.summary()
+    traffic = committed_traffic("attn_fwd", w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w.name, "S": S, "H": H, "d": d, "P": P, "batch": 1,
+                   "q_sigma": w.q_sigma, "kv_sigma": w.kv_sigma,
+                   "step": f"attn_fwd + {P} x attn_fwd_partial + attn_merge",
+                   "step_flops": step_flops,
+                   "l2": f"inputs larger than L2 (Q,K,V {3 * S * H * d * 2 / 2**20:.0f} MiB, "
+                         f"partials {P * S * H * d * 4 / 2**20:.0f} MiB per step)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,false>",
+                     "achieved": mono_tflops, "peak": pk["tc_sustained"], "unit": "TFLOP/s",
+                     "frac": mono_tflops / pk["tc_sustained"],
+                     "frac_of_burst_peak": mono_tflops / pk["tc_burst"],
+                     "peak_source": pk["source"] + "; sustained figure (kernel timed inside a long step)",
+                     "traffic": traffic,
+                     "algorithmic": "4*S^2*d*H flops per launch"},
+        "kernels": {"attn_fwd_ms": mono_ms, "attn_fwd_tflops": mono_tflops,
+                    "partial_pass_ms": part_ms,
+                    "partial_pass_tflops": w.flops / (part_ms * 1e-3) / 1e12,
+                    "merge_ms": merge_ms, "merge_gbs": merge_gbs,
+                    "merge_hbm_frac": merge_gbs / pk["hbm_gbs"], "merge_bytes": merge_bytes},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * (P + 2),
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------- reference arm --
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = W.ATTN_WORKLOADS[args.workload]
+    rows = 8  # query rows per head per step: a bounded sample of the workload
+    for _ in range(args.warmup):
+        oracle_sample(w, rows)
+    total_flops, total_s = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(w, rows)
+        total_flops += f
+        total_s += dt
+    value = total_flops / total_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "S": w.S, "H": w.H, "d": w.d, "P": max(w.P, 1), "batch": 1,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"FP64 numpy oracle, {rows} query rows per head x {w.H} heads "
+                                   f"against all {w.S} keys per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

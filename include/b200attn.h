@@ -1,0 +1,189 @@
+/*
+ * b200attn -- non-causal long-sequence self-attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libb200attn.so.  Plain pointers and sizes only.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - fp16 tensors are passed as uint16_t* holding IEEE binary16 bit patterns.
+ * - "device" pointers must be CUDA device memory of the current device;
+ *   "host" pointers are ordinary (preferably page-locked) host memory.
+ * - Ownership: the caller owns every buffer.  The library allocates no
+ *   device memory on any call path and keeps no pointer after a call returns
+ *   (TMA descriptors are built per call).
+ * - Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as
+ *   void*, NULL = the legacy default stream) and the call returns without
+ *   waiting, except where stated.  Buffers must stay valid until the stream
+ *   reaches the work.
+ * - Errors: every entry point returns a b2a_status.  Arguments are checked
+ *   before anything is enqueued; on B2A_ERR_INVALID_ARG or
+ *   B2A_ERR_UNSUPPORTED nothing was enqueued and no output was touched.
+ *   B2A_ERR_CUDA means a CUDA runtime call failed; b2a_last_cuda_error()
+ *   returns its cudaError_t.  Kernels never trap: a device-side wait that
+ *   runs out (a lost arrival) sets a device status word and the kernel
+ *   returns; b2a_check_status() reports it as B2A_ERR_TIMEOUT.
+ * - Batch is 1.  Token-major layouts follow the pages' (S, B, hidden)
+ *   activations with B = 1 ("Multi-Device Attention Inference with
+ *   TensorRT", Generating the ONNX Models).
+ */
+#ifndef B200ATTN_H
+#define B200ATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define B2A_API __attribute__((visibility("default")))
+#else
+#define B2A_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  B2A_OK = 0,
+  B2A_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, stride or scale */
+  B2A_ERR_UNSUPPORTED = 2, /* not an sm_100 device, or a size beyond an implementation limit */
+  B2A_ERR_CUDA = 3,        /* a CUDA runtime call failed; see b2a_last_cuda_error() */
+  B2A_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (reported by b2a_check_status) */
+} b2a_status;
+
+/*
+ * attn_fwd -- monolithic non-causal scaled-dot-product attention.
+ *
+ * Per head h and query row i (every token attends to every token:
+ * "Multi-Device Attention Inference with TensorRT", Introduction; per-head
+ * attention: "Tensor Parallelism: Sharding Weights for Parallel Layer
+ * Execution", section 3, step 3):
+ *   out[i, h, :] = sum_j softmax_j(scale * q[i,h,:] . k[j,h,:]) * v[j, h, :]
+ *   lse[h, i]    = ln sum_j exp(scale * q[i,h,:] . k[j,h,:])
+ *
+ * q, k, v   device fp16, row-major [S, H, d] with row strides ld_q, ld_k,
+ *           ld_v elements (head h at columns h*d .. h*d+d-1 of a row); for
+ *           views into a fused QKV buffer [S, 3*H*d] pass ld = 3*H*d.
+ * out       device fp16 [S, H, d] with row stride ld_o.
+ * lse       device fp32 [H, S] (natural log, scale included); may be NULL.
+ * S >= 1, H >= 1, d in {64, 128}, scale > 0 and finite.
+ * Every ld >= H*d and a multiple of 8; every pointer 16-byte aligned.
+ * Arithmetic: fp16 products, fp32 accumulation and softmax, P rounded to
+ * fp16 for the P.V product, output rounded once to fp16.
+ */
+B2A_API int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
+             int S, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o, void* stream);
+
+/*
+ * attn_fwd_partial -- attention of all queries against one contiguous chunk
+ * of keys, the per-step work of ring attention (TensorRT 11.0 multi-device
+ * article, the three context-parallel implementations, Ring Attention).
+ *
+ *   o_part[i, h, :] = softmax over the chunk's keys only, times their values
+ *   lse_part[h, i]  = ln sum_{j in chunk} exp(scale * q_i . k_j)
+ *
+ * q         device fp16 [Sq, H, d], row stride ld_q.
+ * k_chunk,
+ * v_chunk   device fp16 [Skv, H, d], row stride ld_kv (pointer offsets into
+ *           the full K/V give the chunk; chunk p of P is conventionally keys
+ *           [floor(p*S/P), floor((p+1)*S/P))).
+ * o_part    device fp32 [Sq, H, d], contiguous (normalised by the chunk's
+ *           own sum).
+ * lse_part  device fp32 [H, Sq].
+ * Sq >= 1, Skv >= 0: an empty chunk writes o_part = 0 and lse_part = -inf.
+ * Other requirements as attn_fwd.
+ */
+B2A_API int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
+                     float* o_part, float* lse_part, int Sq, int Skv, int H, int d, float scale,
+                     int ld_q, int ld_kv, void* stream);
+
+/*
+ * attn_merge -- exact merge of P chunk partials (ring attention's
+ * online-softmax combine; the "split-reduction" of the accuracy table in
+ * "TensorRT Multi-Device (multi-GPU) support", Validation):
+ *   L = max_p lse_p;  lse = L + ln sum_p exp(lse_p - L)
+ *   out = sum_p exp(lse_p - lse) * o_p        (chunks with lse_p = -inf add 0)
+ *
+ * o_parts    device fp32 [P, S, H, d] contiguous (chunk p's o_part at
+ *            offset p*S*H*d).
+ * lse_parts  device fp32 [P, H, S] contiguous.
+ * out        device fp16 [S, H, d] contiguous.
+ * lse_out    device fp32 [H, S]; may be NULL.
+ * 1 <= P <= 64 (B2A_ERR_UNSUPPORTED above), S >= 1, H >= 1, d in {64, 128}.
+ */
+B2A_API int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
+               int S, int H, int d, void* stream);
+
+/*
+ * qkv_proj -- fused Q/K/V projection qkv = x * w_qkv^T ("Tensor Parallelism:
+ * Sharding Weights for Parallel Layer Execution", section 3, step 1:
+ * Q = X W_Q, K = X W_K, V = X W_V, here as one weight).
+ *
+ * x      device fp16 [M, K] row-major.
+ * w_qkv  device fp16 [N, K] row-major ([out, in]); N = 3*H*d with rows
+ *        [W_Q; W_K; W_V], each head-major.
+ * qkv    device fp16 [M, N] row-major.
+ * M, N, K >= 1; N and K multiples of 8; pointers 16-byte aligned.
+ * fp32 accumulation, one rounding to fp16.
+ */
+B2A_API int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, int M, int N, int K,
+             void* stream);
+
+/*
+ * out_proj -- output projection with residual, y = residual + a * w_o^T
+ * (section 3, step 4 of the same lesson: Z = Concat(heads) W_O; the block
+ * adds its input back).  The residual is added to the fp32 accumulator and
+ * the sum is rounded once to fp16.
+ *
+ * a         device fp16 [M, K] (the concatenated head outputs).
+ * w_o       device fp16 [N, K] ([out, in]).
+ * residual  device fp16 [M, N] or NULL (then y = a * w_o^T); may equal y.
+ * y         device fp16 [M, N].
+ * Requirements as qkv_proj.
+ */
+B2A_API int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* residual, uint16_t* y, int M,
+             int N, int K, void* stream);
+
+/*
+ * attn_fwd_host -- attention end to end from host memory.
+ *
+ * Copies q, k, v (host fp16 [S, H, d] contiguous) into the caller's device
+ * workspace, runs attn_fwd (P == 1) or P attn_fwd_partial calls plus
+ * attn_merge (P > 1, the one-device emulation of ring attention), and copies
+ * out (host fp16 [S, H, d]) and lse (host fp32 [H, S], may be NULL) back.
+ * All copies are cudaMemcpyAsync on `stream`; the call returns after
+ * enqueueing, so the host buffers must stay valid until the stream is
+ * synchronised.  With page-locked host buffers the copies are asynchronous.
+ *
+ * workspace        device memory of at least attn_fwd_host_workspace_bytes(S,H,d,P)
+ *                  bytes, 256-byte aligned.
+ * workspace_bytes  its size (checked).
+ * 1 <= P <= 64; other requirements as attn_fwd.
+ */
+B2A_API int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                  float* lse, int S, int H, int d, float scale, int P, void* workspace,
+                  uint64_t workspace_bytes, void* stream);
+
+/* Device workspace attn_fwd_host needs; 0 for invalid sizes. */
+B2A_API uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P);
+
+/*
+ * b2a_check_status -- synchronise `stream`, then read and clear the device
+ * status word that kernels set when a bounded wait runs out.  Returns
+ * B2A_OK, B2A_ERR_TIMEOUT, or B2A_ERR_CUDA if the synchronisation failed.
+ * Blocks the calling host thread.
+ */
+B2A_API int b2a_check_status(void* stream);
+
+/* Static text for a b2a_status value. */
+B2A_API const char* b2a_status_string(int status);
+
+/* cudaError_t of the most recent failed CUDA call in this thread (0 if none). */
+B2A_API int b2a_last_cuda_error(void);
+
+/* Library ABI version (major*100 + minor). */
+B2A_API int b2a_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200ATTN_H */

@@ -1,0 +1,265 @@
+"""Python binding of libb200attn.so: non-causal long-sequence attention on B200.
+
+Argument marshalling only.  Every step of the computation runs in the CUDA
+library; torch tensors supply device memory and the current stream.  There
+is no CPU or eager fallback: if the library is missing or the device is not
+an sm_100 part, calls raise.
+
+Tensor layouts (batch 1):
+  q, k, v, out  fp16 [S, H, d]; rows may be strided (views into a fused QKV
+                buffer), the head and feature dims must be dense.
+  lse           fp32 [H, S], natural log of sum_j exp(scale * q.k_j).
+  o_parts       fp32 [P, S, H, d];  lse_parts fp32 [P, H, S].
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from .build import LIB as _LIB_PATH
+
+__all__ = [
+    "B2AError", "lib", "attn_fwd", "attn_fwd_partial", "attn_merge", "attn_chunked",
+    "qkv_proj", "out_proj", "attn_fwd_host", "host_workspace_bytes", "check_status",
+    "chunk_bounds", "library_path",
+]
+
+B2A_OK, B2A_ERR_INVALID_ARG, B2A_ERR_UNSUPPORTED, B2A_ERR_CUDA, B2A_ERR_TIMEOUT = range(5)
+
+_u16p = ctypes.c_void_p
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+
+_SIGS = {
+    "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _i, _i, _i, _vp]),
+    "attn_fwd_partial": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
+    "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "out_proj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, ctypes.c_uint64, _vp]),
+    "attn_fwd_host_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),
+    "b2a_check_status": (_i, [_vp]),
+    "b2a_status_string": (ctypes.c_char_p, [_i]),
+    "b2a_last_cuda_error": (_i, []),
+    "b2a_version": (_i, []),
+}
+
+
+class B2AError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        msg = lib.b2a_status_string(status).decode()
+        extra = ""
+        if status == B2A_ERR_CUDA:
+            extra = f" (cudaError {lib.b2a_last_cuda_error()})"
+        super().__init__(f"{fn}: {msg}{extra}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"libb200attn.so not found at {_LIB_PATH}; build it with "
+            "`python -m long_context_bidirectional_b200.build` (needs nvcc)")
+    handle = ctypes.CDLL(_LIB_PATH)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(handle, name)
+        fn.restype = res
+        fn.argtypes = args
+    return handle
+
+
+lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(lib, name)(*args)
+    if st != B2A_OK:
+        raise B2AError(name, st)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_qkv(name: str, t: torch.Tensor, H: int | None = None, d: int | None = None) -> int:
+    """Validate an fp16 CUDA [S, H, d] view; return its row stride in elements."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.float16:
+        raise TypeError(f"{name} must be float16, got {t.dtype}")
+    if t.dim() != 3:
+        raise ValueError(f"{name} must be [S, H, d], got shape {tuple(t.shape)}")
+    S_, H_, d_ = t.shape
+    if (H is not None and H_ != H) or (d is not None and d_ != d):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected [*, {H}, {d}]")
+    if t.stride(2) != 1 or (H_ > 1 and t.stride(1) != d_):
+        raise ValueError(f"{name}: head and feature dims must be dense (strides {t.stride()})")
+    return t.stride(0) if S_ > 1 else max(t.stride(0), H_ * d_)
+
+
+def _default_scale(d: int, scale):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def attn_fwd(q, k, v, out=None, lse=None, scale=None, return_lse=True, stream=None):
+    """Monolithic non-causal attention; returns ``(out, lse)`` (lse may be None)."""
+    S, H, d = q.shape
+    ld_q = _check_qkv("q", q)
+    ld_k = _check_qkv("k", k, H, d)
+    ld_v = _check_qkv("v", v, H, d)
+    if k.shape[0] != S or v.shape[0] != S:
+        raise ValueError("attn_fwd is self-attention: q, k, v need the same S")
+    if out is None:
+        out = torch.empty((S, H, d), dtype=torch.float16, device=q.device)
+    ld_o = _check_qkv("out", out, H, d)
+    if lse is None and return_lse:
+        lse = torch.empty((H, S), dtype=torch.float32, device=q.device)
+    _call("attn_fwd", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+          S, H, d, _default_scale(d, scale), ld_q, ld_k, ld_v, ld_o, _stream(stream))
+    return out, lse
+
+
+def attn_fwd_partial(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None, stream=None):
+    """Attention of all queries against one key chunk; returns ``(o_part, lse_part)``."""
+    Sq, H, d = q.shape
+    ld_q = _check_qkv("q", q)
+    Skv = k_chunk.shape[0]
+    ld_k = _check_qkv("k_chunk", k_chunk, H, d)
+    ld_v = _check_qkv("v_chunk", v_chunk, H, d)
+    if v_chunk.shape[0] != Skv:
+        raise ValueError("k_chunk and v_chunk need the same length")
+    if ld_k != ld_v:
+        raise ValueError("k_chunk and v_chunk must share a row stride")
+    if o_part is None:
+        o_part = torch.empty((Sq, H, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((H, Sq), dtype=torch.float32, device=q.device)
+    if not (o_part.is_contiguous() and o_part.dtype == torch.float32 and o_part.numel() == Sq * H * d):
+        raise ValueError("o_part must be contiguous float32 [Sq, H, d]")
+    if not (lse_part.is_contiguous() and lse_part.dtype == torch.float32 and lse_part.numel() == H * Sq):
+        raise ValueError("lse_part must be contiguous float32 [H, Sq]")
+    # An empty chunk may be a zero-length view; any valid address will do.
+    kp = k_chunk.data_ptr() if Skv > 0 else q.data_ptr()
+    vp = v_chunk.data_ptr() if Skv > 0 else q.data_ptr()
+    _call("attn_fwd_partial", q.data_ptr(), kp, vp, o_part.data_ptr(), lse_part.data_ptr(),
+          Sq, Skv, H, d, _default_scale(d, scale), ld_q, ld_k if Skv > 0 else ld_q, _stream(stream))
+    return o_part, lse_part
+
+
+def attn_merge(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stream=None):
+    """Exact merge of partials ``o_parts [P,S,H,d]``, ``lse_parts [P,H,S]``."""
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("o_parts and lse_parts must be float32")
+    if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
+        raise ValueError("o_parts and lse_parts must be contiguous")
+    P, S, H, d = o_parts.shape
+    if tuple(lse_parts.shape) != (P, H, S):
+        raise ValueError(f"lse_parts must be [P, H, S] = {(P, H, S)}, got {tuple(lse_parts.shape)}")
+    if out is None:
+        out = torch.empty((S, H, d), dtype=torch.float16, device=o_parts.device)
+    if not (out.is_contiguous() and out.dtype == torch.float16 and out.numel() == S * H * d):
+        raise ValueError("out must be contiguous float16 [S, H, d]")
+    if lse_out is None and return_lse:
+        lse_out = torch.empty((H, S), dtype=torch.float32, device=o_parts.device)
+    _call("attn_merge", o_parts.data_ptr(), lse_parts.data_ptr(), P, out.data_ptr(), _ptr(lse_out),
+          S, H, d, _stream(stream))
+    return out, lse_out
+
+
+def chunk_bounds(S: int, P: int):
+    """Chunk ``p`` of ``P`` covers keys ``[floor(p*S/P), floor((p+1)*S/P))``."""
+    return [((p * S) // P, ((p + 1) * S) // P) for p in range(P)]
+
+
+def attn_chunked(q, k, v, P: int, out=None, lse=None, scale=None, o_parts=None, lse_parts=None,
+                 stream=None):
+    """Ring attention emulated on one device: P key-chunk partials, then the merge.
+
+    ``o_parts``/``lse_parts`` are the caller's workspace (allocated here when
+    omitted).  Returns ``(out, lse)``.
+    """
+    S, H, d = q.shape
+    if o_parts is None:
+        o_parts = torch.empty((P, S, H, d), dtype=torch.float32, device=q.device)
+    if lse_parts is None:
+        lse_parts = torch.empty((P, H, S), dtype=torch.float32, device=q.device)
+    for c, (lo, hi) in enumerate(chunk_bounds(k.shape[0], P)):
+        attn_fwd_partial(q, k[lo:hi], v[lo:hi], o_parts[c], lse_parts[c], scale=scale, stream=stream)
+    return attn_merge(o_parts, lse_parts, out=out, lse_out=lse, stream=stream)
+
+
+def _check_mat(name, t, rows=None, cols=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.float16:
+        raise TypeError(f"{name} must be a float16 CUDA tensor")
+    if t.dim() != 2 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 2-D tensor")
+    if (rows is not None and t.shape[0] != rows) or (cols is not None and t.shape[1] != cols):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected ({rows}, {cols})")
+
+
+def qkv_proj(x, w_qkv, out=None, stream=None):
+    """``out = x @ w_qkv.T``; x [M, K], w_qkv [N, K] fp16."""
+    M, K = x.shape
+    N = w_qkv.shape[0]
+    _check_mat("x", x)
+    _check_mat("w_qkv", w_qkv, N, K)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check_mat("out", out, M, N)
+    _call("qkv_proj", x.data_ptr(), w_qkv.data_ptr(), out.data_ptr(), M, N, K, _stream(stream))
+    return out
+
+
+def out_proj(a, w_o, residual=None, out=None, stream=None):
+    """``out = residual + a @ w_o.T`` (residual optional, may be ``out``)."""
+    M, K = a.shape
+    N = w_o.shape[0]
+    _check_mat("a", a)
+    _check_mat("w_o", w_o, N, K)
+    if residual is not None:
+        _check_mat("residual", residual, M, N)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=a.device)
+    _check_mat("out", out, M, N)
+    _call("out_proj", a.data_ptr(), w_o.data_ptr(), _ptr(residual), out.data_ptr(), M, N, K,
+          _stream(stream))
+    return out
+
+
+def host_workspace_bytes(S: int, H: int, d: int, P: int) -> int:
+    return int(lib.attn_fwd_host_workspace_bytes(S, H, d, P))
+
+
+def attn_fwd_host(q, k, v, out, lse, workspace, P: int = 1, scale=None, stream=None):
+    """End-to-end call from host memory (pinned CPU tensors), see the C header."""
+    S, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous() or tuple(t.shape) != (S, H, d):
+            raise ValueError(f"{name} must be a contiguous float16 host tensor [S, H, d]")
+    if lse is not None and (lse.is_cuda or lse.dtype != torch.float32 or lse.numel() != H * S):
+        raise ValueError("lse must be a float32 host tensor [H, S]")
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be device memory")
+    _call("attn_fwd_host", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+          S, H, d, _default_scale(d, scale), P, workspace.data_ptr(),
+          workspace.numel() * workspace.element_size(), _stream(stream))
+    return out, lse
+
+
+def check_status(stream=None) -> None:
+    """Synchronise and raise if any kernel reported a device-side timeout."""
+    _call("b2a_check_status", _stream(stream))

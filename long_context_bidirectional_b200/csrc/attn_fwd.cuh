@@ -1,0 +1,404 @@
+// Non-causal flash-style attention forward for sm_100a (tcgen05 + TMEM + TMA).
+//
+// Computes, per head h and query row i, o_i = sum_j softmax_j(scale*q_i.k_j) v_j
+// and the natural-log log-sum-exp of the scaled logits ("Multi-Device
+// Attention Inference with TensorRT", Introduction: every token attends to
+// every token; "Tensor Parallelism: Sharding Weights for Parallel Layer
+// Execution", section 3, step 3: attention per head).  Keys are visited in
+// 128-wide tiles with an online (running-max) softmax, the form ring
+// attention relies on (TensorRT 11.0 multi-device article, Ring Attention).
+//
+// One CTA owns two 128-row query tiles of one head.  Warp roles:
+//   warps 0-3  softmax for query tile 0 (thread = one query row)
+//   warps 4-7  softmax for query tile 1
+//   warp  8    TMA producer (Q once, then K_j, V_j through a smem ring)
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1.  The softmax
+// writes P (fp16, two per column) over the first half of its S block and the
+// PV MMA reads it from there as the A operand.  MMA issue order per key tile
+// j is PV0(j-1.. ) interleaved so that one softmax group always has a tile
+// to work on while the tensor core runs the other group's MMAs:
+//   QK0(0) QK1(0) | PV0(0) QK0(1) PV1(0) QK1(1) | PV0(1) QK0(2) ...
+// A tcgen05.commit tracks every MMA issued before it, so when S_q(j+1) is
+// signalled the PV that last wrote O_q is complete; the softmax thread may
+// then rescale its O row in place (done lazily, only when the running max
+// grows by more than 2^8, which keeps every P value <= 256).
+#pragma once
+
+#include <cmath>
+
+#include "ptx.cuh"
+
+namespace b2a {
+
+struct AttnParams {
+  int Sq;             // query rows
+  int Skv;            // key/value rows
+  int H;              // heads
+  float scale_log2;   // scale * log2(e)
+  uint16_t* out;      // monolithic: fp16 [Sq, ld_o], head h at column h*D
+  int ld_o;
+  float* lse;         // monolithic: fp32 [H, Sq] (nullable)
+  float* o_part;      // partial: fp32 [Sq, H, D]
+  float* lse_part;    // partial: fp32 [H, Sq]
+  unsigned int* status;
+};
+
+template <int D>
+struct AttnShape {
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static constexpr int BM = 128;                  // query rows per tile
+  static constexpr int BN = 128;                  // keys per tile
+  static constexpr int QT = 2;                    // query tiles per CTA
+  static constexpr int SUB = D / 64;              // 128-byte column blocks per row
+  static constexpr int SUB_BYTES = 128 * 128;     // one [128 rows x 128 B] block
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int STAGES = D == 128 ? 4 : 8;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = QT * Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + STAGES * KV_BYTES;
+  // barriers: q_full, kv_full[STAGES], kv_empty[STAGES], s_full[2], p_full[2],
+  //           o_full[2], drain
+  static constexpr int B_Q = 0;
+  static constexpr int B_KVF = 1;
+  static constexpr int B_KVE = 1 + STAGES;
+  static constexpr int B_S = 1 + 2 * STAGES;
+  static constexpr int B_P = B_S + 2;
+  static constexpr int B_O = B_P + 2;
+  static constexpr int B_DRAIN = B_O + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1 KB alignment
+  static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
+  static constexpr int TM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static constexpr int ROWS_PER_CTA = QT * BM;
+};
+
+// Running max is kept in units of log2-scaled logits; P = 2^(t - m) <= 2^8.
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Wait ignoring the abort flag, used only to drain in-flight async work.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+template <int D, bool PARTIAL>
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnShape<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int head = blockIdx.y;
+  const int q0 = blockIdx.x * C::ROWS_PER_CTA;
+  const int nkv = (p.Skv + C::BN - 1) / C::BN;
+
+  const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+  const uint32_t sKV = smem_u32(smem + C::OFF_KV);
+  const uint32_t sBar = smem_u32(smem + C::OFF_BAR);
+  auto bar = [&](int i) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::B_KVF + s), 1);
+      mbar_init(bar(C::B_KVE + s), 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(bar(C::B_S + q), 1);
+      mbar_init(bar(C::B_P + q), 128);
+      mbar_init(bar(C::B_O + q), 1);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(bar(C::B_Q), C::QT * C::Q_BYTES);
+#pragma unroll
+      for (int qt = 0; qt < C::QT; ++qt)
+#pragma unroll
+        for (int sb = 0; sb < C::SUB; ++sb)
+          tma_load_3d(sQ + qt * C::Q_BYTES + sb * C::SUB_BYTES, &tm_q, bar(C::B_Q), sb * 64, head,
+                      q0 + qt * C::BM);
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        for (int kind = 0; kind < 2; ++kind) {
+          const int idx = 2 * j + kind;
+          const int st = idx % C::STAGES;
+          const uint32_t par = ((idx / C::STAGES) & 1) ^ 1;
+          if (!mbar_wait(bar(C::B_KVE + st), par, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::B_KVF + st), C::KV_BYTES);
+          const CUtensorMap* m = kind ? &tm_v : &tm_k;
+#pragma unroll
+          for (int sb = 0; sb < C::SUB; ++sb)
+            tma_load_3d(sKV + st * C::KV_BYTES + sb * C::SUB_BYTES, m, bar(C::B_KVF + st), sb * 64,
+                        head, j * C::BN);
+          ++issued;
+        }
+      }
+      if (!ok) {
+        // Let every copy still in flight land before the CTA can exit.
+        mbar_drain(bar(C::B_Q), 0);
+        for (int idx = issued - C::STAGES; idx < issued; ++idx) {
+          if (idx < 0) continue;
+          mbar_drain(bar(C::B_KVF + idx % C::STAGES), (idx / C::STAGES) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);
+      auto issue_qk = [&](int qt, int st) {
+        const uint32_t d_t = tmem + (qt ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
+          mma_ss(d_t, sw128_desc(sQ + qt * C::Q_BYTES + off, 16, 1024),
+                 sw128_desc(sKV + st * C::KV_BYTES + off, 16, 1024), idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int qt, int st, bool acc) {
+        const uint32_t d_t = tmem + (qt ? C::TM_O1 : C::TM_O0);
+        const uint32_t a_t = tmem + (qt ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk) {
+          // V tile is MN-major (d contiguous): 16 keys = 16 rows of 128 B.
+          mma_ts(d_t, a_t + kk * 8, sw128_desc(sKV + st * C::KV_BYTES + kk * 2048, C::SUB_BYTES, 1024),
+                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto wait_kv = [&](int idx, int& st) -> bool {
+        st = idx % C::STAGES;
+        return mbar_wait(bar(C::B_KVF + st), (idx / C::STAGES) & 1, abort_flag, p.status);
+      };
+      bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, p.status);
+      int stk = 0, stv = 0;
+      if (ok) ok = wait_kv(0, stk);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, stk);
+        tc_commit(bar(C::B_S + 0));
+        issue_qk(1, stk);
+        tc_commit(bar(C::B_S + 1));
+        tc_commit(bar(C::B_KVE + stk));
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const bool more = (j + 1 < nkv);
+        if (!(ok = wait_kv(2 * j + 1, stv))) break;
+        if (!(ok = mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_pv(0, stv, j > 0);
+        if (!more) tc_commit(bar(C::B_O + 0));
+        if (more) {
+          if (!(ok = wait_kv(2 * j + 2, stk))) break;
+          tc_fence_after();
+          issue_qk(0, stk);
+          tc_commit(bar(C::B_S + 0));
+        }
+        if (!(ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_pv(1, stv, j > 0);
+        tc_commit(bar(C::B_KVE + stv));
+        if (!more) tc_commit(bar(C::B_O + 1));
+        if (more) {
+          issue_qk(1, stk);
+          tc_commit(bar(C::B_S + 1));
+          tc_commit(bar(C::B_KVE + stk));
+        }
+      }
+      // Every MMA issued above must finish before TMEM is released.
+      tc_commit(bar(C::B_DRAIN));
+      mbar_drain(bar(C::B_DRAIN), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- softmax --
+    const int qt = warp >> 2;
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (qt ? C::TM_S1 : C::TM_S0);
+    const uint32_t tO = tmem + lane_off + (qt ? C::TM_O1 : C::TM_O0);
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY;  // running max, log2-scaled units
+    float l = 0.f;             // running sum of 2^(t - m_used)
+    bool ok = true;
+
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait_warp(bar(C::B_S + qt), j & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r0[32], r1[32], r2[32], r3[32];
+      tmem_ld32(tS + 0, r0);
+      tmem_ld32(tS + 32, r1);
+      tmem_ld32(tS + 64, r2);
+      tmem_ld32(tS + 96, r3);
+      tmem_wait_ld(r0);
+      tmem_wait_ld(r1);
+      tmem_wait_ld(r2);
+      tmem_wait_ld(r3);
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        s[c] = __uint_as_float(r0[c]);
+        s[32 + c] = __uint_as_float(r1[c]);
+        s[64 + c] = __uint_as_float(r2[c]);
+        s[96 + c] = __uint_as_float(r3[c]);
+      }
+      const int valid = p.Skv - j * C::BN;
+      if (valid < C::BN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * sl2;
+      const float m_new = fmaxf(m_used, m_tile);
+      const bool need = m_new > m_used + kRescaleThreshold;
+      const float factor = need ? ex2_approx(m_used - m_new) : 1.f;
+      if (need) {
+        l *= factor;
+        m_used = m_new;
+      }
+      const float neg_m = -m_used;
+      float sum = 0.f;
+#pragma unroll
+      for (int cb = 0; cb < 128; cb += 32) {
+        // 32 scores -> 16 packed fp16x2 words -> TMEM columns cb/2 .. cb/2+15
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float a0 = ex2_approx(fmaf(s[cb + c], sl2, neg_m));
+          const float a1 = ex2_approx(fmaf(s[cb + c + 1], sl2, neg_m));
+          sum += a0 + a1;
+          pk[c >> 1] = pack_half2(a0, a1);
+        }
+        tmem_st16(tS + (cb >> 1), pk);
+      }
+      l += sum;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O_q(j-1) is complete (its PV was issued before this tile's QK)
+        // and PV_q(j) waits for this thread's p_full arrival below.
+#pragma unroll
+        for (int cb = 0; cb < D; cb += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + cb, o);
+          tmem_wait_ld(o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+          tmem_st32(tO + cb, o);
+        }
+        tmem_wait_st();
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_P + qt));
+    }
+
+    if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), 0, abort_flag, p.status);
+    if (ok) {
+      tc_fence_after();
+      const int row = q0 + qt * C::BM + row_in_tile;
+      const bool live = row < p.Sq;
+      const float inv_l = 1.f / l;
+      const float lse_v = (m_used + lg2_approx(l)) * kLn2;
+#pragma unroll
+      for (int cb = 0; cb < D; cb += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + cb, o);
+        tmem_wait_ld(o);
+        if (live) {
+          if constexpr (PARTIAL) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.o_part + (static_cast<size_t>(row) * p.H + head) * D + cb);
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              dst[c >> 2] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
+                                        __uint_as_float(o[c + 2]) * inv_l,
+                                        __uint_as_float(o[c + 3]) * inv_l);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
+                                                  static_cast<size_t>(head) * D + cb);
+#pragma unroll
+            for (int c = 0; c < 32; c += 8)
+              dst[c >> 3] = make_uint4(
+                  pack_half2(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l),
+                  pack_half2(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l),
+                  pack_half2(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l),
+                  pack_half2(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l));
+          }
+        }
+      }
+      if (live) {
+        if constexpr (PARTIAL) {
+          p.lse_part[static_cast<size_t>(head) * p.Sq + row] = lse_v;
+        } else {
+          if (p.lse) p.lse[static_cast<size_t>(head) * p.Sq + row] = lse_v;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+// Fill for an empty key chunk: o = 0, lse = -inf (the empty sum).
+__global__ void attn_empty_partial_kernel(float* o_part, float* lse_part, size_t n_o, size_t n_lse) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_o; i += stride)
+    o_part[i] = 0.f;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_lse; i += stride)
+    lse_part[i] = -INFINITY;
+}
+
+}  // namespace b2a

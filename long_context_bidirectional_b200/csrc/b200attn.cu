@@ -1,0 +1,423 @@
+// C-ABI implementation of libb200attn.so: argument validation, TMA
+// descriptor encoding, kernel launches.  All kernels live in this single
+// translation unit so that they can name the device status word directly.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "b200attn.h"
+#include "attn_fwd.cuh"
+#include "attn_merge.cuh"
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace {
+
+// Set by kernels when a bounded wait runs out; read and cleared by
+// b2a_check_status().  One word per device (static device memory).
+__device__ unsigned int g_status_word;
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return B2A_ERR_CUDA;
+}
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sm_count = 0;
+  unsigned int* status = nullptr;
+};
+
+std::mutex g_dev_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+// Current device; checks it is an sm_100 part and caches facts about it.
+int current_device(const DeviceInfo** info) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return B2A_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e);
+    di.supported = (major == 10 && minor == 0);
+    di.sm_count = sms;
+    if (di.supported) {
+      void* p = nullptr;
+      if ((e = cudaGetSymbolAddress(&p, g_status_word)) != cudaSuccess) return cuda_fail(e);
+      di.status = static_cast<unsigned int*>(p);
+    }
+    di.probed = true;
+  }
+  if (!di.supported) return B2A_ERR_UNSUPPORTED;
+  *info = &di;
+  return B2A_OK;
+}
+
+// ------------------------------------------------------------ TMA maps ----
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// [rows, H, d] fp16 with row stride ld elements; box = 128 rows x 1 head x 64.
+int attn_map(CUtensorMap* m, const void* base, int d, int H, int rows, int ld) {
+  auto enc = encoder();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(ld) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return B2A_OK;
+}
+
+// [rows, K] fp16 row-major; box = box_rows x 64.
+int gemm_map(CUtensorMap* m, const void* base, int rows, int K, int box_rows) {
+  auto enc = encoder();
+  if (!enc) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return B2A_OK;
+}
+
+// ---------------------------------------------------------- validation ----
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool good_ld(int ld, int H, int d) {
+  return ld > 0 && (ld % 8) == 0 && static_cast<long long>(ld) >= static_cast<long long>(H) * d;
+}
+
+inline bool good_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+int validate_attn(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int d,
+                  float scale, int ld_q, int ld_k, int ld_v) {
+  if (!q || !k || !v) return B2A_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return B2A_ERR_INVALID_ARG;
+  if (Sq < 1 || Skv < 0 || H < 1) return B2A_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return B2A_ERR_INVALID_ARG;
+  if (!good_scale(scale)) return B2A_ERR_INVALID_ARG;
+  if (!good_ld(ld_q, H, d) || !good_ld(ld_k, H, d) || !good_ld(ld_v, H, d)) return B2A_ERR_INVALID_ARG;
+  if (H > 65535) return B2A_ERR_UNSUPPORTED;  // grid.y
+  return B2A_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, bool PARTIAL>
+int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int ld_q,
+                int ld_k, int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
+  using C = b2a::AttnShape<D>;
+  CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = attn_map(&tq, q, D, H, Sq, ld_q)) != B2A_OK) return st;
+  if ((st = attn_map(&tk, k, D, H, Skv, ld_k)) != B2A_OK) return st;
+  if ((st = attn_map(&tv, v, D, H, Skv, ld_v)) != B2A_OK) return st;
+  prm.Sq = Sq;
+  prm.Skv = Skv;
+  prm.H = H;
+  prm.scale_log2 = scale * kLog2e;
+  auto kern = b2a::attn_fwd_kernel<D, PARTIAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  dim3 grid((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, H);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return B2A_OK;
+}
+
+int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
+                  int S, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
+                  cudaStream_t stream) {
+  int st = validate_attn(q, k, v, S, S, H, d, scale, ld_q, ld_k, ld_v);
+  if (st != B2A_OK) return st;
+  if (!out || !aligned16(out) || !good_ld(ld_o, H, d)) return B2A_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  b2a::AttnParams prm{};
+  prm.out = out;
+  prm.ld_o = ld_o;
+  prm.lse = lse;
+  prm.status = di->status;
+  if (d == 128)
+    return launch_attn<128, false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
+  return launch_attn<64, false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
+}
+
+int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_part,
+                      float* lse_part, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_kv,
+                      cudaStream_t stream) {
+  int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_kv, ld_kv);
+  if (st != B2A_OK) return st;
+  if (!o_part || !lse_part || !aligned16(o_part) || (reinterpret_cast<uintptr_t>(lse_part) & 3u))
+    return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  if (Skv == 0) {
+    const size_t n_o = static_cast<size_t>(Sq) * H * d;
+    const size_t n_l = static_cast<size_t>(Sq) * H;
+    b2a::attn_empty_partial_kernel<<<di->sm_count * 4, 256, 0, stream>>>(o_part, lse_part, n_o, n_l);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+  }
+  b2a::AttnParams prm{};
+  prm.o_part = o_part;
+  prm.lse_part = lse_part;
+  prm.status = di->status;
+  if (d == 128)
+    return launch_attn<128, true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
+  return launch_attn<64, true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
+}
+
+int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
+                    int S, int H, int d, cudaStream_t stream) {
+  if (!o_parts || !lse_parts || !out) return B2A_ERR_INVALID_ARG;
+  if (!aligned16(o_parts) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
+    return B2A_ERR_INVALID_ARG;
+  if (lse_out && (reinterpret_cast<uintptr_t>(lse_out) & 3u)) return B2A_ERR_INVALID_ARG;
+  if (P < 1 || S < 1 || H < 1 || (d != 64 && d != 128)) return B2A_ERR_INVALID_ARG;
+  if (P > b2a::kMergeMaxP) return B2A_ERR_UNSUPPORTED;
+  const long long npairs = static_cast<long long>(S) * H;
+  const long long blocks = (npairs + b2a::kMergePairs - 1) / b2a::kMergePairs;
+  if (blocks > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  const int smem = P * b2a::kMergePairs * static_cast<int>(sizeof(float));
+  cudaError_t e;
+  if (d == 128) {
+    e = cudaFuncSetAttribute(b2a::attn_merge_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    b2a::attn_merge_kernel<128><<<static_cast<unsigned>(blocks), b2a::kMergePairs, smem, stream>>>(
+        o_parts, lse_parts, P, S, H, out, lse_out);
+  } else {
+    e = cudaFuncSetAttribute(b2a::attn_merge_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    b2a::attn_merge_kernel<64><<<static_cast<unsigned>(blocks), b2a::kMergePairs, smem, stream>>>(
+        o_parts, lse_parts, P, S, H, out, lse_out);
+  }
+  e = cudaGetLastError();
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+
+int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t* c, int M, int N, int K,
+              cudaStream_t stream) {
+  if (!a || !w || !c) return B2A_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(c) || (r && !aligned16(r))) return B2A_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || (N % 8) != 0 || (K % 8) != 0) return B2A_ERR_INVALID_ARG;
+  using G = b2a::GemmShape;
+  const long long tiles_m = (M + G::BM - 1) / G::BM;
+  const long long tiles_n = (N + G::BN - 1) / G::BN;
+  if (tiles_m * tiles_n > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  CUtensorMap ta, tb;
+  if ((st = gemm_map(&ta, a, M, K, G::BM)) != B2A_OK) return st;
+  if ((st = gemm_map(&tb, w, N, K, G::BN)) != B2A_OK) return st;
+  b2a::GemmParams prm{};
+  prm.M = M;
+  prm.N = N;
+  prm.K = K;
+  prm.tiles_m = static_cast<int>(tiles_m);
+  prm.tiles_n = static_cast<int>(tiles_n);
+  prm.num_tiles = static_cast<int>(tiles_m * tiles_n);
+  prm.c = c;
+  prm.r = r;
+  prm.status = di->status;
+  cudaError_t e = cudaFuncSetAttribute(b2a::gemm_tn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       G::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int grid = prm.num_tiles < di->sm_count ? prm.num_tiles : di->sm_count;
+  b2a::gemm_tn_kernel<<<grid, G::THREADS, G::SMEM_BYTES, stream>>>(ta, tb, prm);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+
+// Workspace layout of attn_fwd_host: q | k | v | out | lse [| o_parts | lse_parts],
+// each region starting on a 256-byte boundary.
+struct HostWs {
+  uint64_t q, k, v, out, lse, o_parts, lse_parts, total;
+};
+
+inline uint64_t up256(uint64_t x) { return (x + 255u) & ~static_cast<uint64_t>(255u); }
+
+bool host_ws_layout(int S, int H, int d, int P, HostWs* w) {
+  if (S < 1 || H < 1 || (d != 64 && d != 128) || P < 1 || P > b2a::kMergeMaxP) return false;
+  const uint64_t n = static_cast<uint64_t>(S) * H * d;
+  const uint64_t nl = static_cast<uint64_t>(S) * H;
+  uint64_t off = 0;
+  w->q = off; off = up256(off + n * 2);
+  w->k = off; off = up256(off + n * 2);
+  w->v = off; off = up256(off + n * 2);
+  w->out = off; off = up256(off + n * 2);
+  w->lse = off; off = up256(off + nl * 4);
+  w->o_parts = off;
+  w->lse_parts = off;
+  if (P > 1) {
+    w->o_parts = off; off = up256(off + static_cast<uint64_t>(P) * n * 4);
+    w->lse_parts = off; off = up256(off + static_cast<uint64_t>(P) * nl * 4);
+  }
+  w->total = off;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse, int S,
+             int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o, void* stream) {
+  return attn_fwd_impl(q, k, v, out, lse, S, H, d, scale, ld_q, ld_k, ld_v, ld_o,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk, float* o_part,
+                     float* lse_part, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_kv,
+                     void* stream) {
+  return attn_partial_impl(q, k_chunk, v_chunk, o_part, lse_part, Sq, Skv, H, d, scale, ld_q, ld_kv,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S,
+               int H, int d, void* stream) {
+  return attn_merge_impl(o_parts, lse_parts, P, out, lse_out, S, H, d, static_cast<cudaStream_t>(stream));
+}
+
+int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, int M, int N, int K, void* stream) {
+  return gemm_impl(x, w_qkv, nullptr, qkv, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* residual, uint16_t* y, int M, int N,
+             int K, void* stream) {
+  return gemm_impl(a, w_o, residual, y, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P) {
+  HostWs w;
+  return host_ws_layout(S, H, d, P, &w) ? w.total : 0;
+}
+
+int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse, int S,
+                  int H, int d, float scale, int P, void* workspace, uint64_t workspace_bytes,
+                  void* stream_) {
+  if (!q || !k || !v || !out || !workspace) return B2A_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return B2A_ERR_INVALID_ARG;
+  if (P > b2a::kMergeMaxP) return B2A_ERR_UNSUPPORTED;
+  HostWs w;
+  if (!host_ws_layout(S, H, d, P, &w)) return B2A_ERR_INVALID_ARG;
+  if (!good_scale(scale)) return B2A_ERR_INVALID_ARG;
+  if (workspace_bytes < w.total) return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint16_t* dq = reinterpret_cast<uint16_t*>(ws + w.q);
+  uint16_t* dk = reinterpret_cast<uint16_t*>(ws + w.k);
+  uint16_t* dv = reinterpret_cast<uint16_t*>(ws + w.v);
+  uint16_t* dout = reinterpret_cast<uint16_t*>(ws + w.out);
+  float* dlse = reinterpret_cast<float*>(ws + w.lse);
+  const size_t nbytes = static_cast<size_t>(S) * H * d * 2;
+  const size_t lbytes = static_cast<size_t>(S) * H * 4;
+  cudaError_t e;
+  if ((e = cudaMemcpyAsync(dq, q, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemcpyAsync(dk, k, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
+  if ((e = cudaMemcpyAsync(dv, v, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
+  const int ld = H * d;
+  if (P == 1) {
+    st = attn_fwd_impl(dq, dk, dv, dout, dlse, S, H, d, scale, ld, ld, ld, ld, stream);
+  } else {
+    float* op = reinterpret_cast<float*>(ws + w.o_parts);
+    float* lp = reinterpret_cast<float*>(ws + w.lse_parts);
+    const size_t n = static_cast<size_t>(S) * H * d;
+    const size_t nl = static_cast<size_t>(S) * H;
+    st = B2A_OK;
+    for (int c = 0; c < P && st == B2A_OK; ++c) {
+      const long long lo = static_cast<long long>(c) * S / P;
+      const long long hi = static_cast<long long>(c + 1) * S / P;
+      st = attn_partial_impl(dq, dk + lo * ld, dv + lo * ld, op + c * n, lp + c * nl, S,
+                             static_cast<int>(hi - lo), H, d, scale, ld, ld, stream);
+    }
+    if (st == B2A_OK) st = attn_merge_impl(op, lp, P, dout, dlse, S, H, d, stream);
+  }
+  if (st != B2A_OK) return st;
+  if ((e = cudaMemcpyAsync(out, dout, nbytes, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+    return cuda_fail(e);
+  if (lse && (e = cudaMemcpyAsync(lse, dlse, lbytes, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+    return cuda_fail(e);
+  return B2A_OK;
+}
+
+int b2a_check_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  unsigned int v = 0;
+  if ((e = cudaMemcpy(&v, di->status, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess) return cuda_fail(e);
+  if (v == 0) return B2A_OK;
+  const unsigned int zero = 0;
+  if ((e = cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+    return cuda_fail(e);
+  return B2A_ERR_TIMEOUT;
+}
+
+const char* b2a_status_string(int status) {
+  switch (status) {
+    case B2A_OK: return "ok";
+    case B2A_ERR_INVALID_ARG: return "invalid argument";
+    case B2A_ERR_UNSUPPORTED: return "unsupported device or size";
+    case B2A_ERR_CUDA: return "CUDA runtime error";
+    case B2A_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int b2a_last_cuda_error(void) { return t_last_cuda_error; }
+
+int b2a_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,225 @@
+// Projection GEMM for sm_100a: C[M,N] = A[M,K] * W[N,K]^T (+ R[M,N]).
+//
+// The fused QKV projection and the output projection of the self-attention
+// block ("Tensor Parallelism: Sharding Weights for Parallel Layer
+// Execution", section 3: Q = X W_Q, K = X W_K, V = X W_V and
+// Z = Concat(heads) W_O; "Multi-Device Attention Inference with TensorRT",
+// Generating the ONNX Models: Q/K/V and output projections), with weights in
+// the [out, in] layout.  fp16 operands, fp32 accumulation in TMEM, one fp16
+// rounding of (acc + residual) in the epilogue.
+//
+// Persistent kernel, one CTA per SM, 128x256 output tiles, K in steps of 64
+// through a 4-stage TMA ring (128-byte swizzle).  Warp roles:
+//   warp 0     TMA producer
+//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2-5  epilogue (TMEM -> registers -> +residual -> fp16 -> global)
+// The accumulator is double-buffered in TMEM (2 x 256 columns) so the
+// epilogue of tile i overlaps the main loop of tile i+1.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace b2a {
+
+struct GemmParams {
+  int M, N, K;
+  int tiles_m, tiles_n, num_tiles;
+  uint16_t* c;          // [M, N] fp16
+  const uint16_t* r;    // [M, N] fp16 residual (nullable, may alias c)
+  unsigned int* status;
+};
+
+struct GemmShape {
+  static constexpr int BM = 128, BN = 256, BK = 64;
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = BN * BK * 2;   // 32 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  // barriers: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+  static constexpr int B_FULL = 0;
+  static constexpr int B_EMPTY = STAGES;
+  static constexpr int B_ACCF = 2 * STAGES;
+  static constexpr int B_ACCE = 2 * STAGES + 2;
+  static constexpr int B_DRAIN = 2 * STAGES + 4;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int TM_COLS = 512;
+  static constexpr int THREADS = 192;
+  static constexpr int GROUP_M = 16;   // raster: 16 m-blocks share each n sweep
+};
+
+__device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& mb, int& nb) {
+  constexpr int G = GemmShape::GROUP_M;
+  const int per_group = G * p.tiles_n;
+  const int g = tile / per_group;
+  const int first_m = g * G;
+  const int gsize = min(G, p.tiles_m - first_m);
+  const int in = tile - g * per_group;
+  mb = first_m + in % gsize;
+  nb = in / gsize;
+}
+
+__global__ void __launch_bounds__(192, 1)
+    gemm_tn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                   const GemmParams p) {
+  using C = GemmShape;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t sBase = smem_u32(smem);
+  const uint32_t sBar = smem_u32(smem + C::OFF_BAR);
+  auto bar = [&](int i) -> uint32_t { return sBar + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const int nk = (p.K + C::BK - 1) / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar(C::B_FULL + s), 1);
+      mbar_init(bar(C::B_EMPTY + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(C::B_ACCF + b), 1);
+      mbar_init(bar(C::B_ACCE + b), 128);
+    }
+    mbar_init(bar(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        gemm_tile_coords(p, tile, mb, nb);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          if (!mbar_wait(bar(C::B_EMPTY + st), ((it / C::STAGES) & 1) ^ 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::B_FULL + st), C::STAGE_BYTES);
+          const uint32_t sa = sBase + st * C::STAGE_BYTES;
+          tma_load_2d(sa, &tm_a, bar(C::B_FULL + st), kb * C::BK, mb * C::BM);
+          tma_load_2d(sa + C::A_BYTES, &tm_b, bar(C::B_FULL + st), kb * C::BK, nb * C::BN);
+        }
+      }
+      if (!ok) {
+        for (int idx = it - C::STAGES; idx < it; ++idx) {
+          if (idx < 0) continue;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(bar(C::B_FULL + idx % C::STAGES), (idx / C::STAGES) & 1))
+            if (global_timer_ns() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(C::BM, C::BN, false, false);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (!(ok = mbar_wait(bar(C::B_ACCE + buf), ((lt >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        const uint32_t d_t = tmem + buf * C::BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int st = it % C::STAGES;
+          if (!(ok = mbar_wait(bar(C::B_FULL + st), (it / C::STAGES) & 1, abort_flag, p.status))) break;
+          tc_fence_after();
+          const uint32_t sa = sBase + st * C::STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
+            mma_ss(d_t, sw128_desc(sa + kk * 32, 16, 1024), sw128_desc(sa + C::A_BYTES + kk * 32, 16, 1024),
+                   idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(C::B_EMPTY + st));
+        }
+        if (!ok) break;
+        tc_commit(bar(C::B_ACCF + buf));
+      }
+      tc_commit(bar(C::B_DRAIN));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar(C::B_DRAIN), 0))
+        if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
+    __syncwarp();
+  } else {
+    // Epilogue warps 2..5 cover TMEM lane quarters 2,3,0,1.
+    const int quarter = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (!mbar_wait_warp(bar(C::B_ACCF + buf), (lt >> 1) & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      int mb, nb;
+      gemm_tile_coords(p, tile, mb, nb);
+      const int row = mb * C::BM + quarter * 32 + lane;
+      const bool live = row < p.M;
+      const uint32_t t_base = tmem + lane_off + buf * C::BN;
+#pragma unroll 1
+      for (int cb = 0; cb < C::BN; cb += 32) {
+        uint32_t v[32];
+        tmem_ld32(t_base + cb, v);
+        tmem_wait_ld(v);
+        const int col0 = nb * C::BN + cb;
+        if (live) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = col0 + g * 8;
+            if (col < p.N) {
+              const size_t off = static_cast<size_t>(row) * p.N + col;
+              float add[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+              if (p.r) {
+                const uint4 rv = *reinterpret_cast<const uint4*>(p.r + off);
+                const __half2* rh = reinterpret_cast<const __half2*>(&rv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float2 f = __half22float2(rh[e]);
+                  add[2 * e] = f.x;
+                  add[2 * e + 1] = f.y;
+                }
+              }
+              uint4 o;
+              o.x = pack_half2(__uint_as_float(v[g * 8 + 0]) + add[0], __uint_as_float(v[g * 8 + 1]) + add[1]);
+              o.y = pack_half2(__uint_as_float(v[g * 8 + 2]) + add[2], __uint_as_float(v[g * 8 + 3]) + add[3]);
+              o.z = pack_half2(__uint_as_float(v[g * 8 + 4]) + add[4], __uint_as_float(v[g * 8 + 5]) + add[5]);
+              o.w = pack_half2(__uint_as_float(v[g * 8 + 6]) + add[6], __uint_as_float(v[g * 8 + 7]) + add[7]);
+              *reinterpret_cast<uint4*>(p.c + off) = o;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_ACCE + buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+}  // namespace b2a

@@ -1,0 +1,46 @@
+"""Comparison metrics and tolerances for CUDA-vs-oracle parity.
+
+Bars (fp16 inputs, fp32 accumulation, compared with the FP64 oracle):
+  max_abs  = max |gpu - ref|                      <= 4e-3
+  rel_fro  = ||gpu - ref||_F / ||ref||_F          <= 1e-3
+  max |gpu_lse - ref_lse|                          <= 1e-3
+"""
+import numpy as np
+
+MAX_ABS = 4e-3
+REL_FRO = 1e-3
+LSE_ABS = 1e-3
+
+
+def metrics(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    diff = gpu - ref
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    den = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(diff)) / den if den > 0 else float(np.linalg.norm(diff))
+    return max_abs, rel
+
+
+def assert_out_close(gpu, ref, what="out", max_abs=MAX_ABS, rel_fro=REL_FRO):
+    assert np.all(np.isfinite(np.asarray(gpu, dtype=np.float64))), f"{what}: non-finite values"
+    ma, rf = metrics(gpu, ref)
+    assert ma <= max_abs and rf <= rel_fro, f"{what}: max_abs={ma:.3e} rel_fro={rf:.3e}"
+    return ma, rf
+
+
+def assert_lse_close(gpu, ref, what="lse", tol=LSE_ABS):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    both_inf = np.isneginf(gpu) & np.isneginf(ref)
+    d = np.where(both_inf, 0.0, np.abs(gpu - ref))
+    m = float(np.max(d)) if d.size else 0.0
+    assert m <= tol, f"{what}: max |dLSE| = {m:.3e}"
+    return m
+
+
+def fp16_ulp(x):
+    """Spacing of fp16 numbers at |x| (subnormal spacing below 2^-14)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return 2.0 ** (e - 10)
