@@ -143,6 +143,29 @@ B2A_API int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* res
              int N, int K, void* stream);
 
 /*
+ * attn_block_fwd -- one self-attention block of the stacked model:
+ *   qkv = x * w_qkv^T;  a = attention(q, k, v) per head;  y = x + a * w_o^T
+ * (the sample's block of Q/K/V projections, scaled dot-product attention and
+ * output projection: "Multi-Device Attention Inference with TensorRT",
+ * Generating the ONNX Models; six of them stacked: "TensorRT Multi-Device
+ * (multi-GPU) support", Validation, multi-layer model).  Runs qkv_proj,
+ * attn_fwd on strided views of qkv (ld = 3*H*d) and out_proj with the
+ * residual, in that order on `stream`.
+ *
+ * x        device fp16 [S, H*d] (block input; also the residual).
+ * w_qkv    device fp16 [3*H*d, H*d] ([out, in]; rows [W_Q; W_K; W_V]).
+ * w_o      device fp16 [H*d, H*d] ([out, in]).
+ * y        device fp16 [S, H*d]; may equal x (in-place block).
+ * qkv_ws   device fp16 [S, 3*H*d] workspace (holds q|k|v after the call).
+ * attn_ws  device fp16 [S, H*d] workspace (holds the attention output).
+ * Requirements as attn_fwd and qkv_proj; workspaces must not overlap x, y
+ * or each other.
+ */
+B2A_API int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o, uint16_t* y,
+                           uint16_t* qkv_ws, uint16_t* attn_ws, int S, int H, int d, float scale,
+                           void* stream);
+
+/*
  * attn_fwd_host -- attention end to end from host memory.
  *
  * Copies q, k, v (host fp16 [S, H, d] contiguous) into the caller's device

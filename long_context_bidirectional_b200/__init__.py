@@ -19,11 +19,12 @@ import os
 
 import torch
 
-from .build import LIB as _LIB_PATH
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libb200attn.so")
 
 __all__ = [
     "B2AError", "lib", "attn_fwd", "attn_fwd_partial", "attn_merge", "attn_chunked",
-    "qkv_proj", "out_proj", "attn_fwd_host", "host_workspace_bytes", "check_status",
+    "qkv_proj", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
+    "host_workspace_bytes", "check_status",
     "chunk_bounds", "library_path",
 ]
 
@@ -39,6 +40,7 @@ _SIGS = {
     "attn_fwd_partial": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
+    "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "out_proj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, ctypes.c_uint64, _vp]),
     "attn_fwd_host_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),
@@ -52,10 +54,11 @@ _SIGS = {
 class B2AError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        msg = lib.b2a_status_string(status).decode()
+        lib_ = _get_lib()
+        msg = lib_.b2a_status_string(status).decode()
         extra = ""
         if status == B2A_ERR_CUDA:
-            extra = f" (cudaError {lib.b2a_last_cuda_error()})"
+            extra = f" (cudaError {lib_.b2a_last_cuda_error()})"
         super().__init__(f"{fn}: {msg}{extra}")
 
 
@@ -72,7 +75,21 @@ def _load() -> ctypes.CDLL:
     return handle
 
 
-lib = _load()
+_lib = None
+
+
+def _get_lib() -> ctypes.CDLL:
+    """Load libb200attn.so on first use; raises ImportError if it is missing."""
+    global _lib
+    if _lib is None:
+        _lib = _load()
+    return _lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _get_lib()
+    raise AttributeError(name)
 
 
 def library_path() -> str:
@@ -80,7 +97,7 @@ def library_path() -> str:
 
 
 def _call(name: str, *args) -> None:
-    st = getattr(lib, name)(*args)
+    st = getattr(_get_lib(), name)(*args)
     if st != B2A_OK:
         raise B2AError(name, st)
 
@@ -240,8 +257,50 @@ def out_proj(a, w_o, residual=None, out=None, stream=None):
     return out
 
 
+def attn_block_fwd(x, w_qkv, w_o, H: int, d: int, out=None, qkv_ws=None, attn_ws=None, scale=None,
+                   stream=None):
+    """One block: ``out = x + attention(split(x @ w_qkv.T)) @ w_o.T``; ``out`` may be ``x``."""
+    S, h = x.shape
+    if h != H * d:
+        raise ValueError(f"x has {h} columns, expected H*d = {H * d}")
+    _check_mat("x", x)
+    _check_mat("w_qkv", w_qkv, 3 * h, h)
+    _check_mat("w_o", w_o, h, h)
+    if out is None:
+        out = torch.empty_like(x)
+    _check_mat("out", out, S, h)
+    if qkv_ws is None:
+        qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device=x.device)
+    if attn_ws is None:
+        attn_ws = torch.empty((S, h), dtype=torch.float16, device=x.device)
+    _check_mat("qkv_ws", qkv_ws, S, 3 * h)
+    _check_mat("attn_ws", attn_ws, S, h)
+    _call("attn_block_fwd", x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), out.data_ptr(),
+          qkv_ws.data_ptr(), attn_ws.data_ptr(), S, H, d, _default_scale(d, scale), _stream(stream))
+    return out
+
+
+def stack_forward(x, weights, H: int, d: int, scale=None, stream=None, keep=False):
+    """Apply the blocks ``weights = [(w_qkv, w_o), ...]`` in order.
+
+    Returns the final activations, or with ``keep=True`` the list of
+    per-block ``(y, qkv, attn)`` (copies of the workspaces after each block).
+    """
+    S, h = x.shape
+    qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device=x.device)
+    attn_ws = torch.empty((S, h), dtype=torch.float16, device=x.device)
+    cur = x.clone()
+    kept = []
+    for w_qkv, w_o in weights:
+        attn_block_fwd(cur, w_qkv, w_o, H, d, out=cur, qkv_ws=qkv_ws, attn_ws=attn_ws, scale=scale,
+                       stream=stream)
+        if keep:
+            kept.append((cur.clone(), qkv_ws.clone(), attn_ws.clone()))
+    return kept if keep else cur
+
+
 def host_workspace_bytes(S: int, H: int, d: int, P: int) -> int:
-    return int(lib.attn_fwd_host_workspace_bytes(S, H, d, P))
+    return int(_get_lib().attn_fwd_host_workspace_bytes(S, H, d, P))
 
 
 def attn_fwd_host(q, k, v, out, lse, workspace, P: int = 1, scale=None, stream=None):

@@ -86,6 +86,30 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA/ALU pipes, for x <= 8 (Cody-Waite range reduction, then a
+// degree-3 polynomial for 2^f on [-1/2, 1/2] whose coefficients come from
+// the Remez fit in fit_exp2_poly.py; max relative error 7.5e-5, below the
+// fp16 rounding that P receives).  x is clamped at -126 so that the exponent
+// arithmetic stays in range; 2^-126 rounds to 0 in fp16.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;              // 1.5 * 2^23: rounds x to an integer n
+  const float n = t - 12582912.f;
+  const float f = x - n;                       // f in [-1/2, 1/2]
+  float p = 0.0551716685295105f;
+  p = fmaf(p, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  // low bits of t hold n; shifting them into the exponent field scales by 2^n
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Wait ignoring the abort flag, used only to drain in-flight async work.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
@@ -94,7 +118,8 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <int D, bool PARTIAL>
+// EMU: of every 16 score columns, how many take exp2_poly instead of MUFU.
+template <int D, bool PARTIAL, int EMU>
 __global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -129,7 +154,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(C::B_O + q), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
-    *abort_flag = 0;
+    // A CTA launched after an earlier one timed out does no work.
+    *abort_flag = (*reinterpret_cast<volatile unsigned int*>(p.status) != 0u) ? 1 : 0;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -294,9 +320,18 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      // row max: four independent 3-input max chains, then combine
+      float ma = s[0], mb = s[1], mc = s[2], md = s[3];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int c = 4; c < 124; c += 8) {
+        ma = fmax3(ma, s[c], s[c + 1]);
+        mb = fmax3(mb, s[c + 2], s[c + 3]);
+        mc = fmax3(mc, s[c + 4], s[c + 5]);
+        md = fmax3(md, s[c + 6], s[c + 7]);
+      }
+      ma = fmax3(ma, s[124], s[125]);
+      mb = fmax3(mb, s[126], s[127]);
+      const float mx = fmax3(ma, mb, fmaxf(mc, md));
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
@@ -306,21 +341,23 @@ __global__ void __launch_bounds__(320, 1)
         m_used = m_new;
       }
       const float neg_m = -m_used;
-      float sum = 0.f;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int cb = 0; cb < 128; cb += 32) {
         // 32 scores -> 16 packed fp16x2 words -> TMEM columns cb/2 .. cb/2+15
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float a0 = ex2_approx(fmaf(s[cb + c], sl2, neg_m));
-          const float a1 = ex2_approx(fmaf(s[cb + c + 1], sl2, neg_m));
-          sum += a0 + a1;
+          const float x0 = fmaf(s[cb + c], sl2, neg_m);
+          const float x1 = fmaf(s[cb + c + 1], sl2, neg_m);
+          const float a0 = ((c & 15) >= 16 - EMU) ? exp2_poly(x0) : ex2_approx(x0);
+          const float a1 = ((c & 15) + 1 >= 16 - EMU) ? exp2_poly(x1) : ex2_approx(x1);
+          sum[(c >> 1) & 3] += a0 + a1;
           pk[c >> 1] = pack_half2(a0, a1);
         }
         tmem_st16(tS + (cb >> 1), pk);
       }
-      l += sum;
+      l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O_q(j-1) is complete (its PV was issued before this tile's QK)
         // and PV_q(j) waits for this thread's p_full arrival below.

@@ -68,26 +68,44 @@ __global__ void __launch_bounds__(kMergePairs)
   const size_t plane4 = static_cast<size_t>(npairs) * U;  // float4 per chunk
   uint2* dst = reinterpret_cast<uint2*>(out) + pair0 * U;
 
-  for (int u = t; u < units; u += kMergePairs) {
-    const int pi = u / U;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // Two units per thread per pass, all their chunk loads issued before use,
+  // so each thread keeps up to 16 independent 16-byte loads in flight.
+  for (int u0 = t; u0 < units; u0 += 2 * kMergePairs) {
+    const int u1 = u0 + kMergePairs;
+    const bool has1 = u1 < units;
+    const int pi0 = u0 / U;
+    const int pi1 = has1 ? u1 / U : pi0;
+    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc1 = acc0;
     for (int q0 = 0; q0 < P; q0 += 8) {
-      float4 x[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (q0 + i < P) x[i] = __ldcs(src + (q0 + i) * plane4 + u);
+      float4 x0[8], x1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (q0 + i < P) {
-          const float w = w_s[(q0 + i) * kMergePairs + pi];
-          acc.x = fmaf(w, x[i].x, acc.x);
-          acc.y = fmaf(w, x[i].y, acc.y);
-          acc.z = fmaf(w, x[i].z, acc.z);
-          acc.w = fmaf(w, x[i].w, acc.w);
+          x0[i] = __ldcs(src + (q0 + i) * plane4 + u0);
+          if (has1) x1[i] = __ldcs(src + (q0 + i) * plane4 + u1);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (q0 + i < P) {
+          const float w0 = w_s[(q0 + i) * kMergePairs + pi0];
+          acc0.x = fmaf(w0, x0[i].x, acc0.x);
+          acc0.y = fmaf(w0, x0[i].y, acc0.y);
+          acc0.z = fmaf(w0, x0[i].z, acc0.z);
+          acc0.w = fmaf(w0, x0[i].w, acc0.w);
+          if (has1) {
+            const float w1 = w_s[(q0 + i) * kMergePairs + pi1];
+            acc1.x = fmaf(w1, x1[i].x, acc1.x);
+            acc1.y = fmaf(w1, x1[i].y, acc1.y);
+            acc1.z = fmaf(w1, x1[i].z, acc1.z);
+            acc1.w = fmaf(w1, x1[i].w, acc1.w);
+          }
         }
       }
     }
-    dst[u] = make_uint2(pack_half2(acc.x, acc.y), pack_half2(acc.z, acc.w));
+    dst[u0] = make_uint2(pack_half2(acc0.x, acc0.y), pack_half2(acc0.z, acc0.w));
+    if (has1) dst[u1] = make_uint2(pack_half2(acc1.x, acc1.y), pack_half2(acc1.z, acc1.w));
   }
 }
 

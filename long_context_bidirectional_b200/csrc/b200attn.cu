@@ -143,6 +143,11 @@ int validate_attn(const void* q, const void* k, const void* v, int Sq, int Skv, 
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Columns (of every 16) whose exponential runs on the FMA pipe.
+#ifndef B2A_ATTN_EMU
+#define B2A_ATTN_EMU 0
+#endif
+
 template <int D, bool PARTIAL>
 int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int ld_q,
                 int ld_k, int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
@@ -156,7 +161,7 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   prm.Skv = Skv;
   prm.H = H;
   prm.scale_log2 = scale * kLog2e;
-  auto kern = b2a::attn_fwd_kernel<D, PARTIAL>;
+  auto kern = b2a::attn_fwd_kernel<D, PARTIAL, B2A_ATTN_EMU>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   dim3 grid((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, H);
@@ -332,6 +337,22 @@ int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, int M, int
 int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* residual, uint16_t* y, int M, int N,
              int K, void* stream) {
   return gemm_impl(a, w_o, residual, y, M, N, K, static_cast<cudaStream_t>(stream));
+}
+
+int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o, uint16_t* y,
+                   uint16_t* qkv_ws, uint16_t* attn_ws, int S, int H, int d, float scale, void* stream_) {
+  if (!x || !w_qkv || !w_o || !y || !qkv_ws || !attn_ws) return B2A_ERR_INVALID_ARG;
+  if (S < 1 || H < 1 || (d != 64 && d != 128) || !good_scale(scale)) return B2A_ERR_INVALID_ARG;
+  const long long h = static_cast<long long>(H) * d;
+  if (3 * h > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const int hi = static_cast<int>(h);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  int st = gemm_impl(x, w_qkv, nullptr, qkv_ws, S, 3 * hi, hi, stream);
+  if (st != B2A_OK) return st;
+  st = attn_fwd_impl(qkv_ws, qkv_ws + h, qkv_ws + 2 * h, attn_ws, nullptr, S, H, d, scale, 3 * hi, 3 * hi,
+                     3 * hi, hi, stream);
+  if (st != B2A_OK) return st;
+  return gemm_impl(attn_ws, w_o, x, y, S, hi, hi, stream);
 }
 
 uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P) {

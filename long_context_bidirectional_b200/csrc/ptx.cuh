@@ -67,16 +67,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to ``hint_ns`` for the phase.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of ``bar`` with parity ``parity`` to complete.
 // ``abort_flag`` (shared memory) lets one role that gave up release the
 // others quickly.  Returns false on timeout or abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* status) {
+  if (*abort_flag) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t it = 1;; ++it) {
+    // sleeps until the phase completes or ~0.1 ms pass
+    if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (*abort_flag) return false;
+    // Another CTA that gave up releases this one too (the status word is
+    // sticky until the host reads it).
+    if (*reinterpret_cast<volatile unsigned int*>(status) != 0u) {
+      *abort_flag = 1;
+      return false;
+    }
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
       atomicOr(status, kDevErrTimeout);

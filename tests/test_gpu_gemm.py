@@ -1,10 +1,11 @@
 """CUDA projection GEMMs (qkv_proj, out_proj) against the FP64 oracle.
 
-The GPU rounds fp32 accumulators once to fp16; the oracle's exact product is
-rounded by the same rule.  Each element may differ from the exact value by
-half an fp16 ulp of rounding plus the fp32 accumulation error, so the
-per-element bound is one fp16 ulp of the exact value (or 1e-6 near zero),
-on top of the benchmark spec max_abs / rel-Frobenius bars.
+The GPU accumulates fp16 products in fp32 and rounds once to fp16.  Each
+element may differ from the exact product by the final rounding (at most one
+fp16 ulp of the exact value, allowing for a result that rounds across a
+power of two) plus the fp32 summation error, bounded by the standard
+K * 2^-24 * sum_k |a_k w_k| (Higham, Accuracy and Stability of Numerical
+Algorithms, section 3.1).  The max_abs / rel-Frobenius bars apply on top.
 """
 import numpy as np
 import pytest
@@ -23,12 +24,12 @@ def b2a():
     return m
 
 
-def check(gpu16, exact, what):
+def check(gpu16, exact, what, abs_sum, K):
     gpu = np.asarray(gpu16, dtype=np.float64)
     err = np.abs(gpu - exact)
-    bound = np.maximum(fp16_ulp(exact), 1e-6)
+    bound = fp16_ulp(exact) + K * 2.0 ** -24 * abs_sum
     worst = float(np.max(err / bound))
-    assert worst <= 1.0, f"{what}: worst error {worst:.2f} ulp"
+    assert worst <= 1.0, f"{what}: worst error {worst:.2f} of the bound"
     assert_out_close(gpu, exact, what)
 
 
@@ -38,7 +39,7 @@ def test_qkv_proj_shapes(b2a, M, N, K):
     a, w = W.gemm_operands(M, N, K, seed=M + N + K)
     out = b2a.qkv_proj(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda())
     b2a.check_status()
-    check(out.cpu().numpy(), OS.linear(a, w), f"qkv {M}x{N}x{K}")
+    check(out.cpu().numpy(), OS.linear(a, w), f"qkv {M}x{N}x{K}", OS.linear(np.abs(a), np.abs(w)), K)
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (300, 512, 256), (1000, 4096, 4096)])
@@ -48,7 +49,8 @@ def test_out_proj_with_residual(b2a, M, N, K):
     rd = torch.from_numpy(r).cuda()
     y = b2a.out_proj(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda(), residual=rd)
     b2a.check_status()
-    check(y.cpu().numpy(), r.astype(np.float64) + OS.linear(a, w), f"out {M}x{N}x{K}")
+    check(y.cpu().numpy(), r.astype(np.float64) + OS.linear(a, w), f"out {M}x{N}x{K}",
+          OS.linear(np.abs(a), np.abs(w)), K)
     # in place: residual aliases the output
     y2 = rd.clone()
     b2a.out_proj(torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda(), residual=y2, out=y2)
@@ -64,4 +66,5 @@ def test_qkv_proj_full_size_sampled_rows(b2a):
     out = b2a.qkv_proj(torch.from_numpy(x).cuda(), torch.from_numpy(w_qkv).cuda())
     b2a.check_status()
     rows = W.sample_rows(w.S, 1, 0, seed=3)
-    check(out.cpu().numpy()[rows], OS.linear(x[rows], w_qkv), "qkv 32768x12288x4096 sampled")
+    check(out.cpu().numpy()[rows], OS.linear(x[rows], w_qkv), "qkv 32768x12288x4096 sampled",
+          OS.linear(np.abs(x[rows]), np.abs(w_qkv)), w.hidden)

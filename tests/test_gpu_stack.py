@@ -1,0 +1,77 @@
+"""CUDA stacked self-attention blocks against the FP64 oracle.
+
+Both sides start from the same seeded x and weights and round to fp16 at the
+same tensor boundaries (qkv, attention output, block output); nothing the
+GPU computes is fed to the oracle.  One-ulp rounding flips at those
+boundaries are expected (fp32 vs fp64 sums), so each compared tensor must
+meet rel_fro <= 1e-3 and, per element, |gpu - ref| <= max(4e-3, one fp16
+ulp of ref) when both sides start from identical inputs (block 1).  In the
+end-to-end run a flip persists along the residual stream and each block can
+add one more; a flipped q, k or v element also moves the softmax weights of
+near-tied keys.  So every tensor of block i (1-based) is allowed i ulps, and
+rel_fro <= 1e-3 holds throughout.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import stack as OS
+from parity import REL_FRO, MAX_ABS, fp16_ulp, metrics
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def b2a():
+    import long_context_bidirectional_b200 as m
+    return m
+
+
+def measure(gpu16, ref16, ulps=1):
+    gpu = np.asarray(gpu16, dtype=np.float64)
+    ref = np.asarray(ref16, dtype=np.float64)
+    assert np.all(np.isfinite(gpu))
+    err = np.abs(gpu - ref)
+    bound = np.maximum(MAX_ABS, ulps * fp16_ulp(ref))
+    ma, rf = metrics(gpu, ref)
+    return float(np.max(err / bound)), ma, rf
+
+
+def check(gpu16, ref16, what, ulps=1):
+    worst, ma, rf = measure(gpu16, ref16, ulps)
+    assert worst <= 1.0 and rf <= REL_FRO, f"{what}: worst {worst:.2f} of bound, max_abs={ma:.3e} rel_fro={rf:.3e}"
+
+
+def test_stack6_s2048_end_to_end(b2a):
+    w = W.STACK6_S2048
+    x = W.stack_x(w)
+    weights = [W.stack_weights(w, i) for i in range(w.blocks)]
+    ref = OS.stack(x, weights, w.H, w.d, w.scale)
+    wd = [(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()) for a, b in weights]
+    kept = b2a.stack_forward(torch.from_numpy(x).cuda(), wd, w.H, w.d, scale=w.scale, keep=True)
+    b2a.check_status()
+    report, ok = [], True
+    for i, ((y, qkv, a), (ry, rqkv, ra)) in enumerate(zip(kept, ref)):
+        for name, g, r in (("qkv", qkv, rqkv), ("attention", a, ra), ("output", y, ry)):
+            worst, ma, rf = measure(g.cpu().numpy(), r, ulps=i + 1)
+            report.append(f"block {i + 1} {name}: {worst:.2f} of bound, max_abs={ma:.3e} rel_fro={rf:.3e}")
+            ok &= worst <= 1.0 and rf <= REL_FRO
+    assert ok, "\n".join(report)
+
+
+def test_block1_s32768_sampled_rows(b2a):
+    w = W.STACK6
+    x = W.stack_x(w)
+    w_qkv, w_o = W.stack_weights(w, 0)
+    xd = torch.from_numpy(x).cuda()
+    qkv_ws = torch.empty((w.S, 3 * w.hidden), dtype=torch.float16, device="cuda")
+    attn_ws = torch.empty((w.S, w.hidden), dtype=torch.float16, device="cuda")
+    y = b2a.attn_block_fwd(xd, torch.from_numpy(w_qkv).cuda(), torch.from_numpy(w_o).cuda(), w.H, w.d,
+                           qkv_ws=qkv_ws, attn_ws=attn_ws, scale=w.scale)
+    b2a.check_status()
+    rows = W.sample_rows(w.S, 1, 0, seed=7)
+    ry, rqkv, ra = OS.block_rows(x, w_qkv, w_o, w.H, w.d, w.scale, rows)
+    check(qkv_ws.cpu().numpy()[rows], rqkv, "block 1 qkv (sampled rows)")
+    check(attn_ws.cpu().numpy()[rows], ra, "block 1 attention (sampled rows)")
+    check(y.cpu().numpy()[rows], ry, "block 1 output (sampled rows)")
