@@ -8,21 +8,29 @@
 // 128-wide tiles with an online (running-max) softmax, the form ring
 // attention relies on (TensorRT 11.0 multi-device article, Ring Attention).
 //
-// One CTA owns two 128-row query tiles of one head.  Warp roles:
-//   warps 0-3  softmax for query tile 0 (thread = one query row)
-//   warps 4-7  softmax for query tile 1
-//   warp  8    TMA producer (Q once, then K_j, V_j through a smem ring)
-//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+// One CTA owns two 128-row query tiles of one head.  Warp roles (18 warps):
+//   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1.  Each
+//               row is shared by two threads (warps w and w+4 of a group, the
+//               same TMEM lane quarter), each owning 64 of the tile's 128
+//               score columns; the two exchange their row max through shared
+//               memory with a 64-thread named barrier.
+//   warp  16    TMA producer (Q once, then K_j, V_j through a smem ring)
+//   warp  17    TMEM allocator and single-thread tcgen05.mma issuer
 // TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1.  The softmax
 // writes P (fp16, two per column) over the first half of its S block and the
 // PV MMA reads it from there as the A operand.  MMA issue order per key tile
-// j is PV0(j-1.. ) interleaved so that one softmax group always has a tile
-// to work on while the tensor core runs the other group's MMAs:
+// j interleaves the two query tiles so that one softmax group works while
+// the tensor core runs the other group's MMAs:
 //   QK0(0) QK1(0) | PV0(0) QK0(1) PV1(0) QK1(1) | PV0(1) QK0(2) ...
 // A tcgen05.commit tracks every MMA issued before it, so when S_q(j+1) is
-// signalled the PV that last wrote O_q is complete; the softmax thread may
-// then rescale its O row in place (done lazily, only when the running max
-// grows by more than 2^8, which keeps every P value <= 256).
+// signalled the PV that last wrote O_q is complete; the softmax may then
+// rescale its O row in place (done lazily, only when the running max grows
+// by more than 2^8, which keeps every P value <= 256).
+//
+// The tile stays 128 keys wide on purpose: QK^T MMAs of N = 128 read their
+// shared-memory operands at exactly the 128 B/clk the tensor core's
+// shared-memory path delivers; narrower tiles oversubscribe it, and then
+// every mbarrier operation issued meanwhile stalls behind the MMA reads.
 #pragma once
 
 #include <cmath>
@@ -50,6 +58,8 @@ struct AttnShape {
   static constexpr int BM = 128;                  // query rows per tile
   static constexpr int BN = 128;                  // keys per tile
   static constexpr int QT = 2;                    // query tiles per CTA
+  static constexpr int HALF = BN / 2;             // score columns per softmax thread
+  static constexpr int OH = D / 2;                // output columns per softmax thread
   static constexpr int SUB = D / 64;              // 128-byte column blocks per row
   static constexpr int SUB_BYTES = 128 * 128;     // one [128 rows x 128 B] block
   static constexpr int Q_BYTES = BM * D * 2;
@@ -68,17 +78,48 @@ struct AttnShape {
   static constexpr int B_O = B_P + 2;
   static constexpr int B_DRAIN = B_O + 2;
   static constexpr int NBAR = B_DRAIN + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // row-max exchange: [tile][parity][half][row] floats, then the final row
+  // sums: [tile][row] floats
+  static constexpr int OFF_RED = OFF_BAR + NBAR * 8;
+  static constexpr int OFF_LSUM = OFF_RED + QT * 2 * 2 * BM * 4;
+  static constexpr int OFF_MISC = OFF_LSUM + QT * BM * 4;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1 KB alignment
   static constexpr int TM_S0 = 0, TM_S1 = 128, TM_O0 = 256, TM_O1 = 256 + D;
   static constexpr int TM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int SOFTMAX_WARPS = 16;
+  static constexpr int WARP_TMA = 16, WARP_MMA = 17;
+  static constexpr int THREADS = 18 * 32;
   static constexpr int ROWS_PER_CTA = QT * BM;
 };
 
 // Running max is kept in units of log2-scaled logits; P = 2^(t - m) <= 2^8.
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
+
+// Optional per-tile event trace (build with -DB2A_TRACE): one CTA records
+// SM clock stamps of each role's events into g_attn_trace[event][tile].
+enum AttnTraceEvent : int {
+  kTrSReady0 = 0, kTrLdDone0, kTrMaxDone0, kTrPDone0,    // softmax, query tile 0
+  kTrSReady1, kTrLdDone1, kTrMaxDone1, kTrPDone1,        // softmax, query tile 1
+  kTrPv0Issue, kTrQk0Issue, kTrPv1Issue, kTrQk1Issue,    // MMA issuer
+  kTrKLoad, kTrVLoad,                                    // TMA producer
+  kTrPv0Done, kTrPv1Done,                                // MMA issuer, PV issued
+  kTrSlotWait, kTrSlotReady,                             // MMA issuer, K/V slot wait
+  kTrEvents
+};
+constexpr int kTraceTiles = 512;
+#ifdef B2A_TRACE
+__device__ unsigned long long g_attn_trace[kTrEvents][kTraceTiles];
+__device__ int g_attn_trace_cta[2];
+#define B2A_TR(ev, j)                                                                   \
+  do {                                                                                  \
+    if (tracing && (j) < kTraceTiles) g_attn_trace[(ev)][(j)] = clock64();             \
+  } while (0)
+#else
+#define B2A_TR(ev, j) \
+  do {                \
+  } while (0)
+#endif
 
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
@@ -118,9 +159,29 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// 64-thread named barrier for the two warps that share rows (ids 1..8).
+__device__ __forceinline__ void pair_barrier(int id) {
+  asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory");
+}
+
+// Same barrier, returning the AND of both warps' ``v``: the pair agrees on
+// whether to go on, so neither can be left waiting in bar.sync alone.
+__device__ __forceinline__ bool pair_barrier_and(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, 64, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
 // EMU: of every 16 score columns, how many take exp2_poly instead of MUFU.
 template <int D, bool PARTIAL, int EMU>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -134,6 +195,9 @@ __global__ void __launch_bounds__(320, 1)
   const int head = blockIdx.y;
   const int q0 = blockIdx.x * C::ROWS_PER_CTA;
   const int nkv = (p.Skv + C::BN - 1) / C::BN;
+#ifdef B2A_TRACE
+  const bool tracing = blockIdx.x == g_attn_trace_cta[0] && blockIdx.y == g_attn_trace_cta[1];
+#endif
 
   const uint32_t sQ = smem_u32(smem + C::OFF_Q);
   const uint32_t sKV = smem_u32(smem + C::OFF_KV);
@@ -150,15 +214,16 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int q = 0; q < 2; ++q) {
       mbar_init(bar(C::B_S + q), 1);
-      mbar_init(bar(C::B_P + q), 128);
+      mbar_init(bar(C::B_P + q), 8);  // one elected arrival per softmax warp of the tile
       mbar_init(bar(C::B_O + q), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
-    // A CTA launched after an earlier one timed out does no work.
+    // A CTA launched after an earlier one timed out gives up at its first
+    // wait that does not complete at once.
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(p.status) != 0u) ? 1 : 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
     tmem_relinquish();
   }
@@ -167,7 +232,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == C::WARP_TMA) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -192,6 +257,7 @@ __global__ void __launch_bounds__(320, 1)
             break;
           }
           mbar_arrive_expect_tx(bar(C::B_KVF + st), C::KV_BYTES);
+          B2A_TR(kind ? kTrVLoad : kTrKLoad, j);
           const CUtensorMap* m = kind ? &tm_v : &tm_k;
 #pragma unroll
           for (int sb = 0; sb < C::SUB; ++sb)
@@ -210,18 +276,21 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == C::WARP_MMA) {
     // ------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);
+      const uint64_t dq = sw128_desc(sQ, 16, 1024);                 // Q, K-major
+      const uint64_t dk = sw128_desc(sKV, 16, 1024);                // K, K-major
+      const uint64_t dv = sw128_desc(sKV, C::SUB_BYTES, 1024);      // V, MN-major
       auto issue_qk = [&](int qt, int st) {
         const uint32_t d_t = tmem + (qt ? C::TM_S1 : C::TM_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
-          mma_ss(d_t, sw128_desc(sQ + qt * C::Q_BYTES + off, 16, 1024),
-                 sw128_desc(sKV + st * C::KV_BYTES + off, 16, 1024), idesc_qk, kk > 0);
+          mma_ss(d_t, dq + ((qt * C::Q_BYTES + off) >> 4), dk + ((st * C::KV_BYTES + off) >> 4), idesc_qk,
+                 kk > 0);
         }
       };
       auto issue_pv = [&](int qt, int st, bool acc) {
@@ -230,8 +299,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
           // V tile is MN-major (d contiguous): 16 keys = 16 rows of 128 B.
-          mma_ts(d_t, a_t + kk * 8, sw128_desc(sKV + st * C::KV_BYTES + kk * 2048, C::SUB_BYTES, 1024),
-                 idesc_pv, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d_t, a_t + kk * 8, dv + ((st * C::KV_BYTES + kk * 2048) >> 4), idesc_pv,
+                 (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto wait_kv = [&](int idx, int& st) -> bool {
@@ -254,23 +323,29 @@ __global__ void __launch_bounds__(320, 1)
         if (!(ok = wait_kv(2 * j + 1, stv))) break;
         if (!(ok = mbar_wait(bar(C::B_P + 0), j & 1, abort_flag, p.status))) break;
         tc_fence_after();
+        B2A_TR(kTrPv0Issue, j);
         issue_pv(0, stv, j > 0);
         if (!more) tc_commit(bar(C::B_O + 0));
+        B2A_TR(kTrPv0Done, j);
         if (more) {
           if (!(ok = wait_kv(2 * j + 2, stk))) break;
           tc_fence_after();
           issue_qk(0, stk);
           tc_commit(bar(C::B_S + 0));
+          B2A_TR(kTrQk0Issue, j);
         }
         if (!(ok = mbar_wait(bar(C::B_P + 1), j & 1, abort_flag, p.status))) break;
         tc_fence_after();
+        B2A_TR(kTrPv1Issue, j);
         issue_pv(1, stv, j > 0);
         tc_commit(bar(C::B_KVE + stv));
         if (!more) tc_commit(bar(C::B_O + 1));
+        B2A_TR(kTrPv1Done, j);
         if (more) {
           issue_qk(1, stk);
           tc_commit(bar(C::B_S + 1));
           tc_commit(bar(C::B_KVE + stk));
+          B2A_TR(kTrQk1Issue, j);
         }
       }
       // Every MMA issued above must finish before TMEM is released.
@@ -280,58 +355,73 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- softmax --
-    const int qt = warp >> 2;
-    const int quarter = warp & 3;
+    const int qt = warp >> 3;               // query tile
+    const int half = (warp >> 2) & 1;       // which 64 of the 128 score columns
+    const int quarter = warp & 3;           // TMEM lane quarter
     const int row_in_tile = quarter * 32 + lane;
+    const int pair_id = 1 + qt * 4 + quarter;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + (qt ? C::TM_S1 : C::TM_S0);
-    const uint32_t tO = tmem + lane_off + (qt ? C::TM_O1 : C::TM_O0);
+    const uint32_t tO = tmem + lane_off + (qt ? C::TM_O1 : C::TM_O0) + half * C::OH;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED) + qt * (2 * 2 * C::BM);
+    float* lsum = reinterpret_cast<float*>(smem + C::OFF_LSUM) + qt * C::BM;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY;  // running max, log2-scaled units
-    float l = 0.f;             // running sum of 2^(t - m_used)
+    float m_used = -INFINITY;  // running max, log2-scaled units (same in both halves)
+    float l = 0.f;             // this half's running sum of 2^(t - m_used)
     bool ok = true;
+    const bool tr_me = (quarter == 0 && half == 0 && lane == 0);
+    (void)tr_me;
 
     for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait_warp(bar(C::B_S + qt), j & 1, abort_flag, p.status)) {
-        ok = false;
-        break;
-      }
+      // A failed wait still runs the (harmless) TMEM reads below so that the
+      // pair reaches its barrier together; the barrier then stops both.
+      const bool got = mbar_wait_warp(bar(C::B_S + qt), j & 1, abort_flag, p.status);
       tc_fence_after();
-      uint32_t r0[32], r1[32], r2[32], r3[32];
-      tmem_ld32(tS + 0, r0);
-      tmem_ld32(tS + 32, r1);
-      tmem_ld32(tS + 64, r2);
-      tmem_ld32(tS + 96, r3);
+      if (tr_me) B2A_TR(qt ? kTrSReady1 : kTrSReady0, j);
+      uint32_t r0[32], r1[32];
+      tmem_ld32(tS + half * C::HALF + 0, r0);
+      tmem_ld32(tS + half * C::HALF + 32, r1);
       tmem_wait_ld(r0);
       tmem_wait_ld(r1);
-      tmem_wait_ld(r2);
-      tmem_wait_ld(r3);
-      float s[128];
+      if (tr_me) B2A_TR(qt ? kTrLdDone1 : kTrLdDone0, j);
+      float s[64];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         s[c] = __uint_as_float(r0[c]);
         s[32 + c] = __uint_as_float(r1[c]);
-        s[64 + c] = __uint_as_float(r2[c]);
-        s[96 + c] = __uint_as_float(r3[c]);
       }
-      const int valid = p.Skv - j * C::BN;
-      if (valid < C::BN) {
+      const int valid = p.Skv - j * C::BN - half * C::HALF;
+      if (valid < C::HALF) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= valid) s[c] = -INFINITY;
       }
-      // row max: four independent 3-input max chains, then combine
+      // this half's row max: four independent 3-input max chains
       float ma = s[0], mb = s[1], mc = s[2], md = s[3];
 #pragma unroll
-      for (int c = 4; c < 124; c += 8) {
+      for (int c = 4; c < 60; c += 8) {
         ma = fmax3(ma, s[c], s[c + 1]);
         mb = fmax3(mb, s[c + 2], s[c + 3]);
         mc = fmax3(mc, s[c + 4], s[c + 5]);
         md = fmax3(md, s[c + 6], s[c + 7]);
       }
-      ma = fmax3(ma, s[124], s[125]);
-      mb = fmax3(mb, s[126], s[127]);
-      const float mx = fmax3(ma, mb, fmaxf(mc, md));
+      ma = fmax3(ma, s[60], s[61]);
+      mb = fmax3(mb, s[62], s[63]);
+      const float mx_half = fmax3(ma, mb, fmaxf(mc, md));
+      // exchange with the partner thread of the same row; the slot alternates
+      // with the tile so a fast partner cannot overwrite an unread value
+      float* slot = red + (j & 1) * (2 * C::BM);
+      slot[half * C::BM + row_in_tile] = mx_half;
+      // The barrier also orders both threads' S loads before any P store
+      // below: P of the upper half lands in columns the lower half read.
+      tc_fence_before();
+      if (!pair_barrier_and(pair_id, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float mx = fmaxf(mx_half, slot[(half ^ 1) * C::BM + row_in_tile]);
+      if (tr_me) B2A_TR(qt ? kTrMaxDone1 : kTrMaxDone0, j);
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kRescaleThreshold;
@@ -343,8 +433,8 @@ __global__ void __launch_bounds__(320, 1)
       const float neg_m = -m_used;
       float sum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cb = 0; cb < 128; cb += 32) {
-        // 32 scores -> 16 packed fp16x2 words -> TMEM columns cb/2 .. cb/2+15
+      for (int cb = 0; cb < 64; cb += 32) {
+        // 32 scores -> 16 packed fp16x2 words -> P columns (half*64 + cb)/2 ..
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -355,14 +445,14 @@ __global__ void __launch_bounds__(320, 1)
           sum[(c >> 1) & 3] += a0 + a1;
           pk[c >> 1] = pack_half2(a0, a1);
         }
-        tmem_st16(tS + (cb >> 1), pk);
+        tmem_st16(tS + ((half * C::HALF + cb) >> 1), pk);
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
         // O_q(j-1) is complete (its PV was issued before this tile's QK)
-        // and PV_q(j) waits for this thread's p_full arrival below.
+        // and PV_q(j) waits for this warp's p_full arrival below.
 #pragma unroll
-        for (int cb = 0; cb < D; cb += 32) {
+        for (int cb = 0; cb < C::OH; cb += 32) {
           uint32_t o[32];
           tmem_ld32(tO + cb, o);
           tmem_wait_ld(o);
@@ -370,12 +460,22 @@ __global__ void __launch_bounds__(320, 1)
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
           tmem_st32(tO + cb, o);
         }
-        tmem_wait_st();
       }
       tmem_wait_st();
+      if (tr_me) B2A_TR(qt ? kTrPDone1 : kTrPDone0, j);
       tc_fence_before();
-      mbar_arrive(bar(C::B_P + qt));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::B_P + qt));
     }
+
+    // combine the two halves' row sums
+    if (half == 1) lsum[row_in_tile] = l;
+    pair_barrier(pair_id);
+    if (half == 0) l += lsum[row_in_tile];
+    pair_barrier(pair_id);
+    if (half == 0) lsum[row_in_tile] = l;
+    pair_barrier(pair_id);
+    l = lsum[row_in_tile];
 
     if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), 0, abort_flag, p.status);
     if (ok) {
@@ -385,14 +485,15 @@ __global__ void __launch_bounds__(320, 1)
       const float inv_l = 1.f / l;
       const float lse_v = (m_used + lg2_approx(l)) * kLn2;
 #pragma unroll
-      for (int cb = 0; cb < D; cb += 32) {
+      for (int cb = 0; cb < C::OH; cb += 32) {
         uint32_t o[32];
         tmem_ld32(tO + cb, o);
         tmem_wait_ld(o);
         if (live) {
+          const int col = half * C::OH + cb;
           if constexpr (PARTIAL) {
             float4* dst = reinterpret_cast<float4*>(
-                p.o_part + (static_cast<size_t>(row) * p.H + head) * D + cb);
+                p.o_part + (static_cast<size_t>(row) * p.H + head) * D + col);
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
               dst[c >> 2] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
@@ -400,7 +501,7 @@ __global__ void __launch_bounds__(320, 1)
                                         __uint_as_float(o[c + 3]) * inv_l);
           } else {
             uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
-                                                  static_cast<size_t>(head) * D + cb);
+                                                  static_cast<size_t>(head) * D + col);
 #pragma unroll
             for (int c = 0; c < 32; c += 8)
               dst[c >> 3] = make_uint4(
@@ -411,7 +512,7 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      if (live) {
+      if (live && half == 0) {
         if constexpr (PARTIAL) {
           p.lse_part[static_cast<size_t>(head) * p.Sq + row] = lse_v;
         } else {
@@ -423,7 +524,7 @@ __global__ void __launch_bounds__(320, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }

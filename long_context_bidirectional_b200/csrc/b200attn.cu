@@ -88,14 +88,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// [rows, H, d] fp16 with row stride ld elements; box = 128 rows x 1 head x 64.
-int attn_map(CUtensorMap* m, const void* base, int d, int H, int rows, int ld) {
+// [rows, H, d] fp16 with row stride ld elements; box = box_rows x 1 head x 64.
+int attn_map(CUtensorMap* m, const void* base, int d, int H, int rows, int ld, int box_rows) {
   auto enc = encoder();
   if (!enc) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
                         static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(ld) * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -154,9 +154,9 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   using C = b2a::AttnShape<D>;
   CUtensorMap tq, tk, tv;
   int st;
-  if ((st = attn_map(&tq, q, D, H, Sq, ld_q)) != B2A_OK) return st;
-  if ((st = attn_map(&tk, k, D, H, Skv, ld_k)) != B2A_OK) return st;
-  if ((st = attn_map(&tv, v, D, H, Skv, ld_v)) != B2A_OK) return st;
+  if ((st = attn_map(&tq, q, D, H, Sq, ld_q, C::BM)) != B2A_OK) return st;
+  if ((st = attn_map(&tk, k, D, H, Skv, ld_k, C::BN)) != B2A_OK) return st;
+  if ((st = attn_map(&tv, v, D, H, Skv, ld_v, C::BN)) != B2A_OK) return st;
   prm.Sq = Sq;
   prm.Skv = Skv;
   prm.H = H;
@@ -440,5 +440,19 @@ const char* b2a_status_string(int status) {
 int b2a_last_cuda_error(void) { return t_last_cuda_error; }
 
 int b2a_version(void) { return 100; }
+
+#ifdef B2A_TRACE
+// Trace builds only: choose the traced CTA, then read the event table
+// ([event][tile] SM clock stamps, b2a::kTrEvents x b2a::kTraceTiles).
+__attribute__((visibility("default"))) int b2a_trace_select(int bx, int by) {
+  const int v[2] = {bx, by};
+  cudaError_t e = cudaMemcpyToSymbol(b2a::g_attn_trace_cta, v, sizeof(v));
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+__attribute__((visibility("default"))) int b2a_trace_read(unsigned long long* host) {
+  cudaError_t e = cudaMemcpyFromSymbol(host, b2a::g_attn_trace, sizeof(b2a::g_attn_trace));
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+#endif
 
 }  // extern "C"

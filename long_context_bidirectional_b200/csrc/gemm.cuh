@@ -88,7 +88,8 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(C::B_ACCE + b), 128);
     }
     mbar_init(bar(C::B_DRAIN), 1);
-    // A CTA launched after an earlier one timed out does no work.
+    // A CTA launched after an earlier one timed out gives up at its first
+    // wait that does not complete at once.
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(p.status) != 0u) ? 1 : 0;
     fence_mbar_init();
   }

@@ -80,15 +80,12 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// Bounded wait for the phase of ``bar`` with parity ``parity`` to complete.
-// ``abort_flag`` (shared memory) lets one role that gave up release the
-// others quickly.  Returns false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* status) {
-  if (*abort_flag) return false;
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait: sleep in try_wait, give up after kWaitLimitNs, on
+// this CTA's abort flag, or when another CTA has set the status word.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            unsigned int* status) {
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  while (true) {
     // sleeps until the phase completes or ~0.1 ms pass
     if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
     if (*abort_flag) return false;
@@ -104,6 +101,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
       return false;
     }
   }
+}
+
+// Bounded wait for the phase of ``bar`` with parity ``parity`` to complete.
+// ``abort_flag`` (shared memory) lets one role that gave up release the
+// others quickly.  Returns false on timeout or abort.  The fast path is a
+// single try_wait: an MMA issuer calls this between tensor-core groups, and
+// the tensor pipe only has about one instruction of work queued to hide it.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, status);
 }
 
 // Warp-uniform variant: lane 0 polls, the verdict is broadcast, so that the
