@@ -41,10 +41,11 @@ L2_BYTES = 126 * 2 ** 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=25)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=W.SEQ32K.name, choices=sorted(W.ATTN_WORKLOADS))
+    ap.add_argument("--workload", default=W.SEQ32K.name,
+                    choices=sorted(W.ATTN_WORKLOADS) + sorted(W.STACK_WORKLOADS))
     ap.add_argument("--chunks", type=int, default=None,
                     help="override the workload's number of KV chunks P")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -69,13 +70,20 @@ def dist_setup(n_gpus):
 
 
 def reduce_max(x: float, world: int) -> float:
+    """Max of ``x`` over ranks (the timing rule: the slowest rank sets the time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank: float, max_ms: float) -> float:
+    """Whole-job rate: every rank's units over the slowest rank's time (units/s)."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 def barrier(world):
@@ -286,7 +294,7 @@ def run_ours(args, rank, world, local):
     merge_ms = reduce_max(avg("merge"), world)
 
     step_flops = 2.0 * w.flops
-    value = world * step_flops / (ms * 1e-3) / 1e12
+    value = job_throughput(world, step_flops, ms) / 1e12
     pk = peaks()
     mono_tflops = w.flops / (mono_ms * 1e-3) / 1e12
     merge_bytes = P * S * H * d * 4 + P * H * S * 4 + S * H * d * 2 + H * S * 4
@@ -322,7 +330,7 @@ def run_ours(args, rank, world, local):
         e2e_ms = reduce_max(a.elapsed_time(b) / args.steps, world)
         b2a.check_status(stream)
         n16 = S * H * d * 2
-        e2e = {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        e2e = {"value": job_throughput(world, step_flops, e2e_ms) / 1e12, "unit": UNIT,
                "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 2 * 3 * n16, "d2h_bytes_per_step": 2 * (n16 + H * S * 4),
                "path": "attn_fwd_host(P=1) + attn_fwd_host(P=%d) from pinned host buffers" % P}
@@ -366,10 +374,102 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- stack workload --
+
+def run_stack(args, rank, world, local):
+    """Six stacked self-attention blocks (fused QKV GEMM, attention on strided
+    views, output GEMM + residual) on x [S, H*d]; value counts attention plus
+    both projections."""
+    import torch
+    import long_context_bidirectional_b200 as b2a
+
+    w = W.STACK_WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    S, H, d, h = w.S, w.H, w.d, w.hidden
+    x0 = torch.from_numpy(W.stack_x(w)).to(dev)
+    weights = [tuple(torch.from_numpy(t).to(dev) for t in W.stack_weights(w, i)) for i in range(w.blocks)]
+    x = torch.empty_like(x0)
+    qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device=dev)
+    attn_ws = torch.empty((S, h), dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = []
+
+    def step(record):
+        x.copy_(x0)
+        for w_qkv, w_o in weights:
+            if record:
+                e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                e[0].record(stream)
+            b2a.qkv_proj(x, w_qkv, out=qkv_ws, stream=stream)
+            if record:
+                e[1].record(stream)
+            b2a.attn_fwd(qkv_ws[:, 0:h].view(S, H, d), qkv_ws[:, h:2 * h].view(S, H, d),
+                         qkv_ws[:, 2 * h:].view(S, H, d), out=attn_ws.view(S, H, d), scale=w.scale,
+                         return_lse=False, stream=stream)
+            if record:
+                e[2].record(stream)
+            b2a.out_proj(attn_ws, w_o, residual=x, out=x, stream=stream)
+            if record:
+                e[3].record(stream)
+                ev.append(e)
+
+    for _ in range(args.warmup):
+        step(False)
+    b2a.check_status(stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(bus_id_of(local)) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            step(True)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    b2a.check_status(stream)
+    ms = reduce_max(t0.elapsed_time(t1) / args.steps, world)
+    n = len(ev)
+    qkv_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
+    att_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
+    out_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / n
+    f_att = 4.0 * S * S * d * H
+    f_qkv = 2.0 * S * 3 * h * h
+    f_out = 2.0 * S * h * h
+    step_flops = w.blocks * (f_att + f_qkv + f_out)
+    pk = peaks()
+    line = {
+        "metric": METRIC, "value": job_throughput(world, step_flops, ms) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": {"workload": w.name, "S": S, "H": H, "d": d, "blocks": w.blocks, "batch": 1,
+                   "step": "per block: qkv_proj, attn_fwd on strided views, out_proj + residual",
+                   "step_flops": step_flops, "l2": "inputs larger than L2 (weights 128 MiB per block)",
+                   "parallelism": f"replicas x{world}"},
+        "kernels": {"qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms * 1e-3) / 1e12,
+                    "attn_fwd_ms": att_ms, "attn_fwd_tflops": f_att / (att_ms * 1e-3) / 1e12,
+                    "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms * 1e-3) / 1e12},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,false>",
+                     "achieved": f_att / (att_ms * 1e-3) / 1e12, "peak": pk["tc_burst"], "unit": "TFLOP/s",
+                     "frac": f_att / (att_ms * 1e-3) / 1e12 / pk["tc_burst"], "peak_source": pk["source"],
+                     "traffic": None, "algorithmic": "4*S^2*d*H flops per launch"},
+        "cpu_baseline": None, "e2e": None,
+        "gpu_launches": args.steps * w.blocks * 3,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # --------------------------------------------------------- reference arm --
 
 def run_reference(args, rank, world):
     if rank != 0:
+        return
+    if args.workload not in W.ATTN_WORKLOADS:
+        print(json.dumps({"impl": "reference", "unavailable": "the CPU reference arm covers the attention "
+                          "workloads only"}), flush=True)
         return
     w = W.ATTN_WORKLOADS[args.workload]
     rows = 8  # query rows per head per step: a bounded sample of the workload
@@ -404,7 +504,10 @@ def main():
         return
     rank, world, local = dist_setup(args.gpus)
     try:
-        run_ours(args, rank, world, local)
+        if args.workload in W.STACK_WORKLOADS:
+            run_stack(args, rank, world, local)
+        else:
+            run_ours(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist
