@@ -166,6 +166,37 @@ B2A_API int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint1
                            void* stream);
 
 /*
+ * attn_block_fwd_static -- attn_block_fwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this entry point; it exists for users of
+ * the library.  Some callers cannot call cudaMalloc (or any allocator) on
+ * their inference path: a host application or plugin framework that reserved
+ * the GPU's memory up front and forbids further device allocations, code
+ * that must not block or fail on an allocation in a latency-critical loop,
+ * or a caller in another runtime that can hand over only its own input and
+ * output buffers.  This variant computes exactly what attn_block_fwd does,
+ * but keeps its two intermediates -- qkv [S, 3*H*d] and the attention output
+ * [S, H*d], fp16, 8*S*H*d bytes together -- in one static device array of
+ * 64 MiB inside the library instead of caller workspaces.  It calls no
+ * allocator.
+ *
+ * x, w_qkv, w_o, y, S, H, d, scale, stream: as attn_block_fwd (y may equal x).
+ * Limit: S*H*d <= 8388608 (e.g. S = 2048 at hidden 4096); larger sizes
+ * return B2A_ERR_UNSUPPORTED before anything is enqueued.
+ * Memory: every GPU that loads the library holds the 64 MiB array until the
+ * process exits.
+ * First call: the first call on a device looks up the array's address on
+ * that device (cudaGetSymbolAddress), so make it before any stream capture.
+ * Sharing: every call uses the same array, and it keeps the last call's
+ * contents.  Calls that can overlap on the GPU (other streams, other host
+ * threads) race on it; the caller must order them.  Nothing in the array
+ * needs to start at zero: each call writes both intermediates in full
+ * before reading them.
+ */
+B2A_API int attn_block_fwd_static(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o,
+                                  uint16_t* y, int S, int H, int d, float scale, void* stream);
+
+/*
  * attn_fwd_host -- attention end to end from host memory.
  *
  * Copies q, k, v (host fp16 [S, H, d] contiguous) into the caller's device

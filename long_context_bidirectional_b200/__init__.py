@@ -41,6 +41,7 @@ _SIGS = {
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
+    "attn_block_fwd_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "out_proj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, ctypes.c_uint64, _vp]),
     "attn_fwd_host_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),

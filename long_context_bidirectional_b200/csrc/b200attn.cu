@@ -280,6 +280,32 @@ int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t*
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
 }
 
+// Static scratch of attn_block_fwd_static: qkv [S, 3h] then the attention
+// output [S, h], fp16.  A file-scope device array, so no allocator is called;
+// host code only ever passes its device address (looked up per device).
+constexpr size_t kBlockStaticScratchBytes = size_t(64) << 20;
+__device__ __align__(256) uint8_t g_block_static_scratch[kBlockStaticScratchBytes];
+
+uint8_t* g_block_static_ptr[kMaxDevices] = {};
+
+// Address of the static scratch on the current device (set up once per
+// device, with that device current).
+int block_static_scratch(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return B2A_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_block_static_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_block_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_block_static_ptr[dev] = static_cast<uint8_t*>(ptr);
+  }
+  *out = g_block_static_ptr[dev];
+  return B2A_OK;
+}
+
 // Workspace layout of attn_fwd_host: q | k | v | out | lse [| o_parts | lse_parts],
 // each region starting on a 256-byte boundary.
 struct HostWs {
@@ -353,6 +379,22 @@ int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o
                      3 * hi, hi, stream);
   if (st != B2A_OK) return st;
   return gemm_impl(attn_ws, w_o, x, y, S, hi, hi, stream);
+}
+
+int attn_block_fwd_static(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o, uint16_t* y, int S,
+                          int H, int d, float scale, void* stream) {
+  if (!x || !w_qkv || !w_o || !y) return B2A_ERR_INVALID_ARG;
+  if (S < 1 || H < 1 || (d != 64 && d != 128) || !good_scale(scale)) return B2A_ERR_INVALID_ARG;
+  const uint64_t elems = static_cast<uint64_t>(S) * H * d;
+  const uint64_t qkv_bytes = (elems * 6 + 255) & ~static_cast<uint64_t>(255);
+  if (qkv_bytes + elems * 2 > kBlockStaticScratchBytes) return B2A_ERR_UNSUPPORTED;
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  uint8_t* scratch = nullptr;
+  if ((st = block_static_scratch(&scratch)) != B2A_OK) return st;
+  return attn_block_fwd(x, w_qkv, w_o, y, reinterpret_cast<uint16_t*>(scratch),
+                        reinterpret_cast<uint16_t*>(scratch + qkv_bytes), S, H, d, scale, stream);
 }
 
 uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P) {
