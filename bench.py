@@ -172,6 +172,11 @@ def peaks():
             "source": "fallback (profiling recipe figures)"}
 
 
+def attn_kernel_name(d: int) -> str:
+    """The monolithic attention kernel the library launches for head dim ``d``."""
+    return "attn_pair_kernel<false>" if d == 128 else f"attn_fwd_kernel<{d},false>"
+
+
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -352,7 +357,7 @@ def run_ours(args, rank, world, local):
                    "l2": f"inputs larger than L2 (Q,K,V {3 * S * H * d * 2 / 2**20:.0f} MiB, "
                          f"partials {P * S * H * d * 4 / 2**20:.0f} MiB per step)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,false>",
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(d),
                      "achieved": mono_tflops, "peak": pk["tc_burst"], "unit": "TFLOP/s",
                      "frac": mono_tflops / pk["tc_burst"],
                      "frac_of_sustained_peak": mono_tflops / pk["tc_sustained"],
@@ -450,7 +455,7 @@ def run_stack(args, rank, world, local):
         "kernels": {"qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms * 1e-3) / 1e12,
                     "attn_fwd_ms": att_ms, "attn_fwd_tflops": f_att / (att_ms * 1e-3) / 1e12,
                     "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms * 1e-3) / 1e12},
-        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,false>",
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(d),
                      "achieved": f_att / (att_ms * 1e-3) / 1e12, "peak": pk["tc_burst"], "unit": "TFLOP/s",
                      "frac": f_att / (att_ms * 1e-3) / 1e12 / pk["tc_burst"], "peak_source": pk["source"],
                      "traffic": None, "algorithmic": "4*S^2*d*H flops per launch"},

@@ -8,6 +8,7 @@
 // 128-wide tiles with an online (running-max) softmax, the form ring
 // attention relies on (TensorRT 11.0 multi-device article, Ring Attention).
 //
+// Used for head dim 64 (head dim 128 runs on CTA pairs, attn_pair.cuh).
 // One CTA owns two 128-row query tiles of one head.  Warp roles (18 warps):
 //   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1.  Each
 //               row is shared by two threads (warps w and w+4 of a group, the
@@ -22,10 +23,10 @@
 // j interleaves the two query tiles so that one softmax group works while
 // the tensor core runs the other group's MMAs:
 //   QK0(0) QK1(0) | PV0(0) QK0(1) PV1(0) QK1(1) | PV0(1) QK0(2) ...
-// A tcgen05.commit tracks every MMA issued before it, so when S_q(j+1) is
-// signalled the PV that last wrote O_q is complete; the softmax may then
-// rescale its O row in place (done lazily, only when the running max grows
-// by more than 2^8, which keeps every P value <= 256).
+// A commit after every PV_q(j) (o_done of the query tile) lets the softmax
+// rescale its O row in place once PV_q(j-1) has landed (done lazily, only
+// when the running max grows by more than 2^8, which keeps every P value
+// <= 256).
 //
 // The tile stays 128 keys wide on purpose: QK^T MMAs of N = 128 read their
 // shared-memory operands at exactly the 128 B/clk the tensor core's
@@ -110,10 +111,14 @@ enum AttnTraceEvent : int {
 constexpr int kTraceTiles = 512;
 #ifdef B2A_TRACE
 __device__ unsigned long long g_attn_trace[kTrEvents][kTraceTiles];
+__device__ unsigned long long g_attn_trace_ns[kTrEvents][kTraceTiles];  // %globaltimer
 __device__ int g_attn_trace_cta[2];
 #define B2A_TR(ev, j)                                                                   \
   do {                                                                                  \
-    if (tracing && (j) < kTraceTiles) g_attn_trace[(ev)][(j)] = clock64();             \
+    if (tracing && (j) < kTraceTiles) {                                                 \
+      g_attn_trace[(ev)][(j)] = clock64();                                              \
+      g_attn_trace_ns[(ev)][(j)] = global_timer_ns();                                   \
+    }                                                                                   \
   } while (0)
 #else
 #define B2A_TR(ev, j) \
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(576, 1)
         tc_fence_after();
         B2A_TR(kTrPv0Issue, j);
         issue_pv(0, stv, j > 0);
-        if (!more) tc_commit(bar(C::B_O + 0));
+        tc_commit(bar(C::B_O + 0));  // O_0 holds PV0(0..j)
         B2A_TR(kTrPv0Done, j);
         if (more) {
           if (!(ok = wait_kv(2 * j + 2, stk))) break;
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(576, 1)
         B2A_TR(kTrPv1Issue, j);
         issue_pv(1, stv, j > 0);
         tc_commit(bar(C::B_KVE + stv));
-        if (!more) tc_commit(bar(C::B_O + 1));
+        tc_commit(bar(C::B_O + 1));  // O_1 holds PV1(0..j)
         B2A_TR(kTrPv1Done, j);
         if (more) {
           issue_qk(1, stk);
@@ -414,8 +419,10 @@ __global__ void __launch_bounds__(576, 1)
       slot[half * C::BM + row_in_tile] = mx_half;
       // The barrier also orders both threads' S loads before any P store
       // below: P of the upper half lands in columns the lower half read.
+      // ``ok`` carries a failed O wait of the previous tile into the AND,
+      // so a pair always leaves the loop together.
       tc_fence_before();
-      if (!pair_barrier_and(pair_id, got)) {
+      if (!pair_barrier_and(pair_id, got && ok)) {
         ok = false;
         break;
       }
@@ -449,16 +456,24 @@ __global__ void __launch_bounds__(576, 1)
       }
       l += (sum[0] + sum[1]) + (sum[2] + sum[3]);
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O_q(j-1) is complete (its PV was issued before this tile's QK)
-        // and PV_q(j) waits for this warp's p_full arrival below.
+        // Wait for PV_q(j-1) through the commit issued right behind it (o_done
+        // of this query tile, one phase per key tile: it cannot be a phase
+        // ahead, as PV_q(j) needs this warp's p_full arrival below, nor two
+        // behind, as its commit for PV_q(j-2) precedes that of S_q(j)), then
+        // rescale O_q in place.
+        if (!mbar_wait_warp(bar(C::B_O + qt), (j - 1) & 1, abort_flag, p.status)) {
+          ok = false;  // the pair stops at the next exchange (or after the loop)
+        } else {
+          tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < C::OH; cb += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + cb, o);
-          tmem_wait_ld(o);
+          for (int cb = 0; cb < C::OH; cb += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + cb, o);
+            tmem_wait_ld(o);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
-          tmem_st32(tO + cb, o);
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+            tmem_st32(tO + cb, o);
+          }
         }
       }
       tmem_wait_st();
@@ -477,7 +492,7 @@ __global__ void __launch_bounds__(576, 1)
     pair_barrier(pair_id);
     l = lsum[row_in_tile];
 
-    if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), 0, abort_flag, p.status);
+    if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), (nkv - 1) & 1, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
       const int row = q0 + qt * C::BM + row_in_tile;

@@ -13,6 +13,7 @@
 
 #include "b200attn.h"
 #include "attn_fwd.cuh"
+#include "attn_pair.cuh"
 #include "attn_merge.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
@@ -171,6 +172,33 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   return B2A_OK;
 }
 
+// Head dim 128 runs on CTA pairs (one M = 256 MMA per pair, each SM loading
+// half of every K/V tile); head dim 64 on single CTAs with two query tiles.
+
+template <bool PARTIAL>
+int launch_attn_pair(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int ld_q,
+                     int ld_k, int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
+  using C = b2a::AttnPairShape;
+  CUtensorMap tq, tk, tv;
+  int st;
+  if ((st = attn_map(&tq, q, C::D, H, Sq, ld_q, C::BM)) != B2A_OK) return st;
+  if ((st = attn_map(&tk, k, C::D, H, Skv, ld_k, C::BN / 2)) != B2A_OK) return st;
+  if ((st = attn_map(&tv, v, C::D, H, Skv, ld_v, C::BN)) != B2A_OK) return st;
+  prm.Sq = Sq;
+  prm.Skv = Skv;
+  prm.H = H;
+  prm.scale_log2 = scale * kLog2e;
+  auto kern = b2a::attn_pair_kernel<PARTIAL>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // two CTAs (one cluster) per 256 query rows
+  dim3 grid(2 * ((Sq + C::ROWS_PER_PAIR - 1) / C::ROWS_PER_PAIR), H);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return B2A_OK;
+}
+
 int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
                   int S, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
                   cudaStream_t stream) {
@@ -185,8 +213,7 @@ int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   prm.ld_o = ld_o;
   prm.lse = lse;
   prm.status = di->status;
-  if (d == 128)
-    return launch_attn<128, false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
+  if (d == 128) return launch_attn_pair<false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
   return launch_attn<64, false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
 }
 
@@ -210,8 +237,7 @@ int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, f
   prm.o_part = o_part;
   prm.lse_part = lse_part;
   prm.status = di->status;
-  if (d == 128)
-    return launch_attn<128, true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
+  if (d == 128) return launch_attn_pair<true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
   return launch_attn<64, true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
 }
 
@@ -493,6 +519,10 @@ __attribute__((visibility("default"))) int b2a_trace_select(int bx, int by) {
 }
 __attribute__((visibility("default"))) int b2a_trace_read(unsigned long long* host) {
   cudaError_t e = cudaMemcpyFromSymbol(host, b2a::g_attn_trace, sizeof(b2a::g_attn_trace));
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+__attribute__((visibility("default"))) int b2a_trace_read_ns(unsigned long long* host) {
+  cudaError_t e = cudaMemcpyFromSymbol(host, b2a::g_attn_trace_ns, sizeof(b2a::g_attn_trace_ns));
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
 }
 #endif

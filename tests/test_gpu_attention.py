@@ -76,11 +76,12 @@ def test_chunked_small_and_ragged(b2a, S, H, d, P):
     assert_lse_close(lse, ref_lse)
 
 
-def test_peaked_softmax_forces_rescales(b2a):
+@pytest.mark.parametrize("d", [64, 128])
+def test_peaked_softmax_forces_rescales(b2a, d):
     # Q ~ N(0, 4^2): logits std ~4, the running max keeps growing past the
     # lazy-rescale threshold across key tiles.
-    q, k, v = W.qkv(1500, 2, 128, seed=5, q_sigma=4.0)
-    scale = 1 / math.sqrt(128)
+    q, k, v = W.qkv(1500, 2, d, seed=5, q_sigma=4.0)
+    scale = 1 / math.sqrt(d)
     out, lse = run_mono(b2a, q, k, v, scale)
     ref, ref_lse = OA.attention(q, k, v, scale)
     assert_out_close(out, ref, "peaked out")
@@ -95,8 +96,9 @@ def test_peaked_softmax_forces_rescales(b2a):
     assert_lse_close(lse2, ref_lse2)
 
 
-def test_single_key_and_constant_values(b2a):
-    q, k, v = W.qkv(300, 2, 64, seed=9, Skv=1)
+@pytest.mark.parametrize("d", [64, 128])
+def test_single_key_and_constant_values(b2a, d):
+    q, k, v = W.qkv(300, 2, d, seed=9, Skv=1)
     o, l = b2a.attn_fwd_partial(dev(q), dev(k), dev(v), scale=0.125)
     b2a.check_status()
     np.testing.assert_allclose(host(o), np.repeat(v.astype(np.float32), 300, axis=0), atol=1e-6)
@@ -107,6 +109,18 @@ def test_single_key_and_constant_values(b2a):
     v[:] = v[0:1]
     out, _ = run_mono(b2a, q, k, v, 1 / math.sqrt(128))
     assert_out_close(out, np.repeat(v[0:1].astype(np.float64), 500, axis=0), "constant v")
+
+
+@pytest.mark.parametrize("Sq,Skv,d", [(200, 700, 128), (1000, 64, 128), (300, 1, 128), (130, 515, 64)])
+def test_partial_query_and_key_counts_differ(b2a, Sq, Skv, d):
+    # one rank's queries against a gathered (or a single ring step's) K/V
+    q, k, v = W.qkv(Sq, 2, d, seed=Sq + Skv, Skv=Skv)
+    scale = 1 / math.sqrt(d)
+    o, l = b2a.attn_fwd_partial(dev(q), dev(k), dev(v), scale=scale)
+    b2a.check_status()
+    ref, ref_lse = OA.attention(q, k, v, scale)
+    assert_out_close(host(o), ref, f"partial Sq={Sq} Skv={Skv}")
+    assert_lse_close(host(l), ref_lse)
 
 
 def test_empty_chunk_partial(b2a):
