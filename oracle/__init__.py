@@ -11,7 +11,8 @@ Modules:
   natural-log log-sum-exp, written as the plain definition (full logits row,
   max-subtracted exponentials, sum, divide).
 * ``chunked``   -- the KV-chunked form: one partial (output, LSE) per chunk of
-  keys, then the exact log-sum-exp merge.
+  keys, then the exact log-sum-exp merge; and the ring step that folds one
+  chunk into a running (output, LSE).
 * ``stack``     -- the stacked self-attention block: fused QKV projection,
   attention, output projection and residual add, rounded to fp16 at the
   tensor boundaries the C-ABI stores.

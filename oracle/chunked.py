@@ -17,7 +17,9 @@ Multi-Device (multi-GPU) support", Validation, attributes its FP16 error to):
     lse = L + ln(sum_p exp(lse_p - L))
     o   = sum_p exp(lse_p - lse) * o_p
 
-which equals monolithic attention in exact arithmetic.  An empty chunk has
+which equals monolithic attention in exact arithmetic.  Folding the chunks
+in one at a time with the two-term form of the same merge (``accumulate``)
+is what each ring rank does per step.  An empty chunk has
 ``lse_p = -inf`` and ``o_p = 0`` and contributes nothing.  This module does
 not import ``oracle.attention``'s merge logic (there is none there); it calls
 ``attention`` only to produce each chunk's partial.
@@ -69,6 +71,57 @@ def merge(o_parts, lse_parts):
     coef = np.where(np.isneginf(lse_parts) | ~finite[None], 0.0, coef)
     # o[s, h, :] = sum_p coef[p, h, s] * o_parts[p, s, h, :]
     o = np.einsum("phs,pshd->shd", coef, o_parts)
+    return o, lse
+
+
+def accumulate(o_acc, lse_acc, o_c, lse_c):
+    """One ring step: fold chunk ``(o_c, lse_c)`` into the running ``(o_acc, lse_acc)``.
+
+    The online-softmax update a ring-attention rank applies as each K/V
+    block arrives (TensorRT 11.0 multi-device article, Ring Attention),
+    written as the two-term case of the merge above:
+
+        lse_new = ln(exp(lse_acc) + exp(lse_c))
+        o_new   = exp(lse_acc - lse_new) * o_acc + exp(lse_c - lse_new) * o_c
+
+    ``o_* [S, H, d]``, ``lse_* [H, S]`` (widened to float64).  A row with
+    ``lse_acc = -inf`` has seen no key: its ``o_acc`` is ignored (it may hold
+    anything) and the result is ``(o_c, lse_c)``; an empty chunk
+    (``lse_c = -inf``, its ``o_c`` likewise ignored) leaves the row
+    unchanged.  Returns float64 arrays.
+    """
+    o_acc = np.asarray(o_acc).astype(np.float64)
+    lse_acc = np.asarray(lse_acc).astype(np.float64)
+    o_c = np.asarray(o_c).astype(np.float64)
+    lse_c = np.asarray(lse_c).astype(np.float64)
+    seen_a = ~np.isneginf(lse_acc)
+    seen_c = ~np.isneginf(lse_c)
+    L = np.maximum(lse_acc, lse_c)
+    L_safe = np.where(np.isneginf(L), 0.0, L)
+    ea = np.where(seen_a, np.exp(np.where(seen_a, lse_acc, 0.0) - L_safe), 0.0)
+    ec = np.where(seen_c, np.exp(np.where(seen_c, lse_c, 0.0) - L_safe), 0.0)
+    total = ea + ec
+    any_seen = seen_a | seen_c
+    lse_new = np.where(any_seen, L_safe + np.log(np.where(any_seen, total, 1.0)), -np.inf)
+    wa = np.where(any_seen, ea / np.where(any_seen, total, 1.0), 0.0)   # [H, S]
+    wc = np.where(any_seen, ec / np.where(any_seen, total, 1.0), 0.0)
+    o_a = np.where(seen_a.T[:, :, None], o_acc, 0.0)                    # ignore unseen rows' o_acc
+    o_b = np.where(seen_c.T[:, :, None], o_c, 0.0)                      # and an empty chunk's o_c
+    o_new = wa.T[:, :, None] * o_a + wc.T[:, :, None] * o_b
+    return o_new, lse_new
+
+
+def ring_attention(q, k, v, scale: float, P: int, rows=None):
+    """The per-rank ring loop on one device: start empty, fold the ``P``
+    chunks' partials in order with ``accumulate``."""
+    q = np.asarray(q)
+    H, d = q.shape[1], q.shape[2]
+    R = q.shape[0] if rows is None else len(rows if not isinstance(rows, (list, tuple)) else rows[0])
+    o = np.zeros((R, H, d))
+    lse = np.full((H, R), -np.inf)
+    for lo, hi in chunk_bounds(np.asarray(k).shape[0], P):
+        o_c, lse_c = attention(q, np.asarray(k)[lo:hi], np.asarray(v)[lo:hi], scale, rows=rows)
+        o, lse = accumulate(o, lse, o_c, lse_c)
     return o, lse
 
 

@@ -251,6 +251,61 @@ def test_merge_identities():
     assert np.all(om3 == 0) and np.all(np.isneginf(lm3))
 
 
+# ------------------------------------------------------------ ring step ----
+
+def test_accumulate_hand_case():
+    # lse 0 = ln 2 and ln 6: the new lse is ln 8, the weights 2/8 and 6/8
+    o_acc = np.array([[[1.0, -2.0]]])              # [S=1, H=1, d=2]
+    o_c = np.array([[[5.0, 4.0]]])
+    o, lse = C.accumulate(o_acc, np.array([[math.log(2)]]), o_c, np.array([[math.log(6)]]))
+    np.testing.assert_allclose(lse, [[math.log(8)]], atol=1e-15)
+    np.testing.assert_allclose(o, [[[0.25 * 1 + 0.75 * 5, 0.25 * -2 + 0.75 * 4]]], atol=1e-15)
+
+
+def test_accumulate_empty_sides():
+    rng = np.random.default_rng(17)
+    o_c = rng.standard_normal((3, 2, 4))
+    lse_c = rng.standard_normal((2, 3))
+    junk = np.full((3, 2, 4), np.nan)
+    # nothing seen yet: the chunk's result, whatever o_acc holds
+    o, lse = C.accumulate(junk, np.full((2, 3), -np.inf), o_c, lse_c)
+    np.testing.assert_array_equal(o, o_c)
+    np.testing.assert_array_equal(lse, lse_c)
+    # an empty chunk leaves the running result alone
+    o2, l2 = C.accumulate(o_c, lse_c, junk, np.full((2, 3), -np.inf))
+    np.testing.assert_array_equal(o2, o_c)
+    np.testing.assert_array_equal(l2, lse_c)
+    # both empty: still empty
+    o3, l3 = C.accumulate(junk, np.full((2, 3), -np.inf), junk, np.full((2, 3), -np.inf))
+    assert np.all(np.isneginf(l3)) and np.all(o3 == 0)
+
+
+@pytest.mark.parametrize("P", [1, 2, 3, 7, 61, 70])
+def test_ring_steps_equal_monolithic(P):
+    # includes more chunks than keys (empty steps)
+    q, k, v = rand_qkv(23, 2, 8, seed=18, Skv=61, sigma=4.0)
+    out, lse = A.attention(q, k, v, 0.35)
+    o2, l2 = C.ring_attention(q, k, v, 0.35, P)
+    np.testing.assert_allclose(o2, out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l2, lse, rtol=0, atol=1e-12)
+
+
+def test_ring_step_order_does_not_matter():
+    # non-causal: folding the chunks in any order reaches the same result
+    q, k, v = rand_qkv(9, 1, 6, seed=19, Skv=40, sigma=3.0)
+    o_parts, lse_parts = C.partials(q, k, v, 0.5, 5)
+    fwd = (np.zeros((9, 1, 6)), np.full((1, 9), -np.inf))
+    rev = (np.zeros((9, 1, 6)), np.full((1, 9), -np.inf))
+    for p in range(5):
+        fwd = C.accumulate(*fwd, o_parts[p], lse_parts[p])
+        rev = C.accumulate(*rev, o_parts[4 - p], lse_parts[4 - p])
+    np.testing.assert_allclose(fwd[0], rev[0], atol=1e-13)
+    np.testing.assert_allclose(fwd[1], rev[1], atol=1e-13)
+    om, lm = C.merge(o_parts, lse_parts)
+    np.testing.assert_allclose(fwd[0], om, atol=1e-13)
+    np.testing.assert_allclose(fwd[1], lm, atol=1e-13)
+
+
 # ----------------------------------------------------------------- stack ----
 
 def test_round16_matches_ieee_half_from_struct():
