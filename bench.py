@@ -305,6 +305,36 @@ def run_ours(args, rank, world, local):
     merge_bytes = P * S * H * d * 4 + P * H * S * 4 + S * H * d * 2 + H * S * 4
     merge_gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
 
+    # The ring-step form (attn_fwd_accumulate): the same P chunks folded into
+    # one running fp32 output in place, the last step writing fp16.  Timed
+    # separately from the step; not part of ``value``.
+    o_acc = torch.empty((S, H, d), dtype=torch.float32, device=dev)
+    lse_acc = torch.empty((H, S), dtype=torch.float32, device=dev)
+    out_r = torch.empty_like(out)
+
+    def ring_pass():
+        lse_acc.fill_(float("-inf"))
+        for c, (lo, hi) in enumerate(bounds):
+            b2a.attn_fwd_accumulate(qd, kd[lo:hi], vd[lo:hi], o_acc, lse_acc,
+                                    out_r if c == P - 1 else None, scale=w.scale, stream=stream)
+
+    for _ in range(2):
+        ring_pass()
+    b2a.check_status(stream)
+    barrier(world)
+    torch.cuda.synchronize()
+    ra = torch.cuda.Event(enable_timing=True)
+    rb = torch.cuda.Event(enable_timing=True)
+    n_ring = 5
+    ra.record(stream)
+    for _ in range(n_ring):
+        ring_pass()
+    rb.record(stream)
+    torch.cuda.synchronize()
+    b2a.check_status(stream)
+    ring_ms = reduce_max(ra.elapsed_time(rb) / n_ring, world)
+    del o_acc, lse_acc, out_r
+
     # end to end from pinned host memory through the C-ABI host entry point
     e2e = None
     if not args.no_e2e:
@@ -369,6 +399,9 @@ def run_ours(args, rank, world, local):
                     "partial_pass_ms": part_ms,
                     "partial_pass_tflops": w.flops / (part_ms * 1e-3) / 1e12,
                     "merge_ms": merge_ms, "merge_gbs": merge_gbs,
+                    "ring_pass_ms": ring_ms,
+                    "ring_pass_tflops": w.flops / (ring_ms * 1e-3) / 1e12,
+                    "ring_pass": f"{P} x attn_fwd_accumulate in place (not in value)",
                     "merge_hbm_frac": merge_gbs / pk["hbm_gbs"], "merge_bytes": merge_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -96,6 +96,34 @@ B2A_API int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const u
                      int ld_q, int ld_kv, void* stream);
 
 /*
+ * attn_fwd_accumulate -- one ring-attention step in place: fold the keys of
+ * one chunk into a running result, the way each rank of ring attention
+ * updates its output as K/V blocks arrive (TensorRT 11.0 multi-device
+ * article, the three context-parallel implementations, Ring Attention: an
+ * online softmax over the streamed K/V blocks).  With (o_c, lse_c) the
+ * chunk's attn_fwd_partial result:
+ *   lse_new = ln(exp(lse_acc) + exp(lse_c))
+ *   o_new   = exp(lse_acc - lse_new) * o_acc + exp(lse_c - lse_new) * o_c
+ * computed in the kernel's epilogue without writing o_c anywhere.
+ *
+ * q, k_chunk, v_chunk, Sq, Skv, H, d, scale, ld_q, ld_kv: as attn_fwd_partial.
+ * o_acc    device fp32 [Sq, H, d] contiguous, read and written in place.
+ * lse_acc  device fp32 [H, Sq], read and written in place (natural log).
+ *          -inf marks a row that has seen no key yet: its o_acc is then
+ *          ignored (it may hold anything) and replaced by o_c.  Start a ring
+ *          pass with lse_acc = -inf; o_acc needs no initialisation.
+ * out      device fp16 [Sq, H, d] contiguous, or NULL.  When given it also
+ *          receives the fp16 rounding of o_new (pass it on the last step).
+ *          Rows that have seen no key get 0.
+ * Skv == 0 leaves o_acc and lse_acc unchanged (and still writes out).
+ * After the last of P steps over the chunks of attn_fwd_partial, o_acc and
+ * lse_acc equal attn_merge's result before its fp16 rounding.
+ */
+B2A_API int attn_fwd_accumulate(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
+                                float* o_acc, float* lse_acc, uint16_t* out, int Sq, int Skv, int H, int d,
+                                float scale, int ld_q, int ld_kv, void* stream);
+
+/*
  * attn_merge -- exact merge of P chunk partials (ring attention's
  * online-softmax combine; the "split-reduction" of the accuracy table in
  * "TensorRT Multi-Device (multi-GPU) support", Validation):
@@ -232,6 +260,24 @@ B2A_API const char* b2a_status_string(int status);
 
 /* cudaError_t of the most recent failed CUDA call in this thread (0 if none). */
 B2A_API int b2a_last_cuda_error(void);
+
+/*
+ * b2a_set_attn_kernel / b2a_get_attn_kernel -- which attention kernel the
+ * attention entry points (attn_fwd, attn_fwd_partial, attn_fwd_accumulate,
+ * and those built on them) use for head dim 128.  The pages have no
+ * counterpart; this is a tuning and testing control.
+ *   B2A_ATTN_KERNEL_AUTO    (default) CTA pairs when the call has at least
+ *                           96 key tiles of 128 (Skv > 12160), else single CTAs
+ *   B2A_ATTN_KERNEL_SINGLE  single CTAs, two 128-row query tiles each
+ *   B2A_ATTN_KERNEL_PAIR    two-SM CTA pairs issuing M = 256 MMAs
+ * Both compute the same result (the same arithmetic in the same order per
+ * row).  Head dim 64 always uses single CTAs.  Process-wide; takes effect
+ * for calls made after it returns.  Returns B2A_ERR_INVALID_ARG for any
+ * other value.
+ */
+enum { B2A_ATTN_KERNEL_AUTO = 0, B2A_ATTN_KERNEL_SINGLE = 1, B2A_ATTN_KERNEL_PAIR = 2 };
+B2A_API int b2a_set_attn_kernel(int choice);
+B2A_API int b2a_get_attn_kernel(void);
 
 /* Library ABI version (major*100 + minor). */
 B2A_API int b2a_version(void);

@@ -22,13 +22,16 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libb200attn.so")
 
 __all__ = [
-    "B2AError", "lib", "attn_fwd", "attn_fwd_partial", "attn_merge", "attn_chunked",
+    "B2AError", "lib", "attn_fwd", "attn_fwd_partial", "attn_fwd_accumulate", "attn_merge", "attn_chunked",
+    "attn_ring", "set_attn_kernel", "get_attn_kernel", "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE",
+    "ATTN_KERNEL_PAIR",
     "qkv_proj", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
     "host_workspace_bytes", "check_status",
     "chunk_bounds", "library_path",
 ]
 
 B2A_OK, B2A_ERR_INVALID_ARG, B2A_ERR_UNSUPPORTED, B2A_ERR_CUDA, B2A_ERR_TIMEOUT = range(5)
+ATTN_KERNEL_AUTO, ATTN_KERNEL_SINGLE, ATTN_KERNEL_PAIR = range(3)
 
 _u16p = ctypes.c_void_p
 _vp = ctypes.c_void_p
@@ -38,6 +41,9 @@ _f = ctypes.c_float
 _SIGS = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _i, _i, _i, _vp]),
     "attn_fwd_partial": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_fwd_accumulate": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "b2a_set_attn_kernel": (_i, [_i]),
+    "b2a_get_attn_kernel": (_i, []),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
@@ -176,6 +182,63 @@ def attn_fwd_partial(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None
     _call("attn_fwd_partial", q.data_ptr(), kp, vp, o_part.data_ptr(), lse_part.data_ptr(),
           Sq, Skv, H, d, _default_scale(d, scale), ld_q, ld_k if Skv > 0 else ld_q, _stream(stream))
     return o_part, lse_part
+
+
+def attn_fwd_accumulate(q, k_chunk, v_chunk, o_acc, lse_acc, out=None, scale=None, stream=None):
+    """One ring step in place: fold a key chunk into ``(o_acc [Sq,H,d] fp32, lse_acc [H,Sq])``.
+
+    ``lse_acc = -inf`` marks rows with no keys yet.  ``out`` (fp16, optional)
+    also receives the rounded merged output.  Returns ``(o_acc, lse_acc, out)``.
+    """
+    Sq, H, d = q.shape
+    ld_q = _check_qkv("q", q)
+    Skv = k_chunk.shape[0]
+    ld_k = _check_qkv("k_chunk", k_chunk, H, d)
+    ld_v = _check_qkv("v_chunk", v_chunk, H, d)
+    if v_chunk.shape[0] != Skv:
+        raise ValueError("k_chunk and v_chunk need the same length")
+    if ld_k != ld_v:
+        raise ValueError("k_chunk and v_chunk must share a row stride")
+    if not (o_acc.is_contiguous() and o_acc.dtype == torch.float32 and o_acc.numel() == Sq * H * d):
+        raise ValueError("o_acc must be contiguous float32 [Sq, H, d]")
+    if not (lse_acc.is_contiguous() and lse_acc.dtype == torch.float32 and lse_acc.numel() == H * Sq):
+        raise ValueError("lse_acc must be contiguous float32 [H, Sq]")
+    if out is not None and not (out.is_contiguous() and out.dtype == torch.float16
+                                and out.numel() == Sq * H * d):
+        raise ValueError("out must be contiguous float16 [Sq, H, d]")
+    kp = k_chunk.data_ptr() if Skv > 0 else q.data_ptr()
+    vp = v_chunk.data_ptr() if Skv > 0 else q.data_ptr()
+    _call("attn_fwd_accumulate", q.data_ptr(), kp, vp, o_acc.data_ptr(), lse_acc.data_ptr(), _ptr(out),
+          Sq, Skv, H, d, _default_scale(d, scale), ld_q, ld_k if Skv > 0 else ld_q, _stream(stream))
+    return o_acc, lse_acc, out
+
+
+def attn_ring(q, k, v, P: int, out=None, scale=None, o_acc=None, lse_acc=None, stream=None):
+    """Ring attention's per-rank loop on one device: P accumulate steps over
+    the key chunks, the last one writing the fp16 output.  Returns ``(out, lse_acc)``.
+    """
+    S, H, d = q.shape
+    if o_acc is None:
+        o_acc = torch.empty((S, H, d), dtype=torch.float32, device=q.device)
+    if lse_acc is None:
+        lse_acc = torch.empty((H, S), dtype=torch.float32, device=q.device)
+    lse_acc.fill_(float("-inf"))
+    if out is None:
+        out = torch.empty((S, H, d), dtype=torch.float16, device=q.device)
+    bounds = chunk_bounds(k.shape[0], P)
+    for c, (lo, hi) in enumerate(bounds):
+        attn_fwd_accumulate(q, k[lo:hi], v[lo:hi], o_acc, lse_acc, out if c == P - 1 else None,
+                            scale=scale, stream=stream)
+    return out, lse_acc
+
+
+def set_attn_kernel(choice: int) -> None:
+    """Head-dim-128 kernel choice: ATTN_KERNEL_AUTO / _SINGLE / _PAIR (process-wide)."""
+    _call("b2a_set_attn_kernel", int(choice))
+
+
+def get_attn_kernel() -> int:
+    return int(_get_lib().b2a_get_attn_kernel())
 
 
 def attn_merge(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stream=None):

@@ -45,11 +45,12 @@ struct AttnParams {
   int Skv;            // key/value rows
   int H;              // heads
   float scale_log2;   // scale * log2(e)
-  uint16_t* out;      // monolithic: fp16 [Sq, ld_o], head h at column h*D
+  uint16_t* out;      // monolithic: fp16 [Sq, ld_o], head h at column h*D;
+                      // accumulate: fp16 [Sq, H, D] (ld_o = H*D) or null
   int ld_o;
   float* lse;         // monolithic: fp32 [H, Sq] (nullable)
-  float* o_part;      // partial: fp32 [Sq, H, D]
-  float* lse_part;    // partial: fp32 [H, Sq]
+  float* o_part;      // partial: fp32 [Sq, H, D]; accumulate: running o_acc (in place)
+  float* lse_part;    // partial: fp32 [H, Sq]; accumulate: running lse_acc (in place)
   unsigned int* status;
 };
 
@@ -156,6 +157,108 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// What a launch writes.  kModeFwd: fp16 out + optional lse (attn_fwd);
+// kModePartial: fp32 o_part + lse_part of one key chunk (attn_fwd_partial);
+// kModeAccum: one ring step in place -- the chunk's result is merged into
+// the running fp32 o_acc / lse_acc held in o_part / lse_part (the exact
+// log-sum-exp combine of ring attention's online softmax), optionally also
+// writing the fp16 rounding of the merged output to out.
+enum AttnMode : int { kModeFwd = 0, kModePartial = 1, kModeAccum = 2 };
+
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// The running log-sum-exp of one row in log2 units (accumulate mode only;
+// -inf when no keys have been folded in yet).  Read by every thread of the
+// row before the row-sum exchange, which orders it before the update.
+template <int MODE>
+__device__ __forceinline__ float accum_lse2(const AttnParams& p, int row, int head) {
+  if constexpr (MODE == kModeAccum) {
+    if (row < p.Sq) return p.lse_part[static_cast<size_t>(head) * p.Sq + row] * kLog2eF;
+  }
+  return -INFINITY;
+}
+
+// Epilogue of one softmax thread: its query row, NC output columns from
+// ``col`` (TMEM columns tO .. tO+NC-1 hold the un-normalised O), running
+// max ``m`` (log2 units), row sum ``l`` and, in accumulate mode, the row's
+// running lse ``la`` (log2 units).  Every lane runs the TMEM loads.
+template <int D, int MODE, int NC>
+__device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row, int head, int col, bool write_lse,
+                                              uint32_t tO, float m, float l, float la) {
+  static_assert(NC % 32 == 0, "whole 32-column TMEM loads");
+  const bool live = row < p.Sq;
+  const float lse2 = m + lg2_approx(l);  // this launch's keys, log2 units
+  float wc = 1.f / l;                    // weight of the TMEM accumulator
+  float wa = 0.f;                        // weight of the running output
+  float lse_new2 = lse2;
+  if constexpr (MODE == kModeAccum) {
+    if (la > -INFINITY) {
+      const float mx = fmaxf(la, lse2);
+      const float ea = ex2_approx(la - mx), ec = ex2_approx(lse2 - mx);
+      const float inv = 1.f / (ea + ec);
+      lse_new2 = mx + lg2_approx(ea + ec);
+      wa = ea * inv;
+      wc = ec * inv / l;
+    }
+  }
+#pragma unroll
+  for (int cb = 0; cb < NC; cb += 32) {
+    uint32_t o[32];
+    tmem_ld32(tO + cb, o);
+    tmem_wait_ld(o);
+    if (!live) continue;
+    const int c0 = col + cb;
+    if constexpr (MODE == kModeFwd) {
+      uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
+                                            static_cast<size_t>(head) * D + c0);
+#pragma unroll
+      for (int c = 0; c < 32; c += 8)
+        dst[c >> 3] = make_uint4(pack_half2(__uint_as_float(o[c]) * wc, __uint_as_float(o[c + 1]) * wc),
+                                 pack_half2(__uint_as_float(o[c + 2]) * wc, __uint_as_float(o[c + 3]) * wc),
+                                 pack_half2(__uint_as_float(o[c + 4]) * wc, __uint_as_float(o[c + 5]) * wc),
+                                 pack_half2(__uint_as_float(o[c + 6]) * wc, __uint_as_float(o[c + 7]) * wc));
+    } else {
+      float4* acc = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(row) * p.H + head) * D + c0);
+      float v[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(o[c]) * wc;
+      if constexpr (MODE == kModeAccum) {
+        if (wa > 0.f) {
+          float4 a[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) a[c] = acc[c];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            v[4 * c] = fmaf(wa, a[c].x, v[4 * c]);
+            v[4 * c + 1] = fmaf(wa, a[c].y, v[4 * c + 1]);
+            v[4 * c + 2] = fmaf(wa, a[c].z, v[4 * c + 2]);
+            v[4 * c + 3] = fmaf(wa, a[c].w, v[4 * c + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) acc[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+      if constexpr (MODE == kModeAccum) {
+        if (p.out) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(row) * p.H + head) * D + c0);
+#pragma unroll
+          for (int c = 0; c < 32; c += 8)
+            dst[c >> 3] = make_uint4(pack_half2(v[c], v[c + 1]), pack_half2(v[c + 2], v[c + 3]),
+                                     pack_half2(v[c + 4], v[c + 5]), pack_half2(v[c + 6], v[c + 7]));
+        }
+      }
+    }
+  }
+  if (live && write_lse) {
+    const size_t li = static_cast<size_t>(head) * p.Sq + row;
+    if constexpr (MODE == kModeFwd) {
+      if (p.lse) p.lse[li] = lse2 * kLn2;
+    } else {
+      p.lse_part[li] = lse_new2 * kLn2;
+    }
+  }
+}
+
 // Wait ignoring the abort flag, used only to drain in-flight async work.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
@@ -185,7 +288,7 @@ __device__ __forceinline__ bool pair_barrier_and(int id, bool v) {
 }
 
 // EMU: of every 16 score columns, how many take exp2_poly instead of MUFU.
-template <int D, bool PARTIAL, int EMU>
+template <int D, int MODE, int EMU>
 __global__ void __launch_bounds__(576, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -483,6 +586,10 @@ __global__ void __launch_bounds__(576, 1)
       if (lane == 0) mbar_arrive(bar(C::B_P + qt));
     }
 
+    const int row = q0 + qt * C::BM + row_in_tile;
+    // accumulate mode: both halves read the running lse before the exchange
+    // below, which orders the reads before half 0's update in the epilogue
+    const float la = accum_lse2<MODE>(p, row, head);
     // combine the two halves' row sums
     if (half == 1) lsum[row_in_tile] = l;
     pair_barrier(pair_id);
@@ -495,45 +602,7 @@ __global__ void __launch_bounds__(576, 1)
     if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), (nkv - 1) & 1, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
-      const int row = q0 + qt * C::BM + row_in_tile;
-      const bool live = row < p.Sq;
-      const float inv_l = 1.f / l;
-      const float lse_v = (m_used + lg2_approx(l)) * kLn2;
-#pragma unroll
-      for (int cb = 0; cb < C::OH; cb += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + cb, o);
-        tmem_wait_ld(o);
-        if (live) {
-          const int col = half * C::OH + cb;
-          if constexpr (PARTIAL) {
-            float4* dst = reinterpret_cast<float4*>(
-                p.o_part + (static_cast<size_t>(row) * p.H + head) * D + col);
-#pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              dst[c >> 2] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
-                                        __uint_as_float(o[c + 2]) * inv_l,
-                                        __uint_as_float(o[c + 3]) * inv_l);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
-                                                  static_cast<size_t>(head) * D + col);
-#pragma unroll
-            for (int c = 0; c < 32; c += 8)
-              dst[c >> 3] = make_uint4(
-                  pack_half2(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l));
-          }
-        }
-      }
-      if (live && half == 0) {
-        if constexpr (PARTIAL) {
-          p.lse_part[static_cast<size_t>(head) * p.Sq + row] = lse_v;
-        } else {
-          if (p.lse) p.lse[static_cast<size_t>(head) * p.Sq + row] = lse_v;
-        }
-      }
+      attn_epilogue<D, MODE, C::OH>(p, row, head, half * C::OH, half == 0, tO, m_used, l, la);
     }
   }
 
@@ -542,6 +611,20 @@ __global__ void __launch_bounds__(576, 1)
   if (warp == C::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+// Accumulate step with an empty key chunk: the running state is unchanged;
+// only the optional fp16 output is written (0 for rows that have seen no key).
+__global__ void attn_accum_empty_kernel(const float* o_acc, const float* lse_acc, uint16_t* out, int Sq,
+                                        int H, int D) {
+  const size_t n = static_cast<size_t>(Sq) * H * D;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n; i += stride) {
+    const size_t rh = i / D;  // row * H + head
+    const int row = static_cast<int>(rh / H), head = static_cast<int>(rh % H);
+    const bool seen = lse_acc[static_cast<size_t>(head) * Sq + row] > -INFINITY;
+    out[i] = static_cast<uint16_t>(pack_half2(seen ? o_acc[i] : 0.f, 0.f) & 0xffffu);
   }
 }
 

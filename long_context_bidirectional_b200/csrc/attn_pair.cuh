@@ -85,7 +85,7 @@ struct AttnPairShape {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
 };
 
-template <bool PARTIAL>
+template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
@@ -411,6 +411,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
       if (++pst == C::STAGES) { pst = 0; psph ^= 1; }
     }
 
+    const int row = q0 + row_in_tile;
+    // accumulate mode: both halves read the running lse before the exchange
+    // below, which orders the reads before half 0's update in the epilogue
+    const float la = accum_lse2<MODE>(p, row, head);
     // combine the two halves' row sums
     if (half == 1) lsum[row_in_tile] = l;
     pair_barrier(pair_id);
@@ -423,45 +427,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     if (ok) ok = mbar_wait_warp(bar(C::B_OF), 0, abort_flag, p.status);
     if (ok) {
       tc_fence_after();
-      const int row = q0 + row_in_tile;
-      const bool live = row < p.Sq;
-      const float inv_l = 1.f / l;
-      const float lse_v = (m_used + lg2_approx(l)) * kLn2;
-#pragma unroll
-      for (int cb = 0; cb < C::HALF; cb += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + cb, o);
-        tmem_wait_ld(o);
-        if (live) {
-          const int col = half * C::HALF + cb;
-          if constexpr (PARTIAL) {
-            float4* dst = reinterpret_cast<float4*>(
-                p.o_part + (static_cast<size_t>(row) * p.H + head) * D + col);
-#pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              dst[c >> 2] = make_float4(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l,
-                                        __uint_as_float(o[c + 2]) * inv_l,
-                                        __uint_as_float(o[c + 3]) * inv_l);
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
-                                                  static_cast<size_t>(head) * D + col);
-#pragma unroll
-            for (int c = 0; c < 32; c += 8)
-              dst[c >> 3] = make_uint4(
-                  pack_half2(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l),
-                  pack_half2(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l));
-          }
-        }
-      }
-      if (live && half == 0) {
-        if constexpr (PARTIAL) {
-          p.lse_part[static_cast<size_t>(head) * p.Sq + row] = lse_v;
-        } else {
-          if (p.lse) p.lse[static_cast<size_t>(head) * p.Sq + row] = lse_v;
-        }
-      }
+      attn_epilogue<D, MODE, C::HALF>(p, row, head, half * C::HALF, half == 0, tO, m_used, l, la);
     }
   }
 

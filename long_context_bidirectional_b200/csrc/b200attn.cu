@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -149,7 +150,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 #define B2A_ATTN_EMU 0
 #endif
 
-template <int D, bool PARTIAL>
+template <int D, int MODE>
 int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int ld_q,
                 int ld_k, int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
   using C = b2a::AttnShape<D>;
@@ -162,7 +163,7 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   prm.Skv = Skv;
   prm.H = H;
   prm.scale_log2 = scale * kLog2e;
-  auto kern = b2a::attn_fwd_kernel<D, PARTIAL, B2A_ATTN_EMU>;
+  auto kern = b2a::attn_fwd_kernel<D, MODE, B2A_ATTN_EMU>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   dim3 grid((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, H);
@@ -173,9 +174,23 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
 }
 
 // Head dim 128 runs on CTA pairs (one M = 256 MMA per pair, each SM loading
-// half of every K/V tile); head dim 64 on single CTAs with two query tiles.
+// half of every K/V tile) when a launch has at least kPairMinKeyTiles key
+// tiles; shorter key ranges and head dim 64 run on single CTAs with two
+// query tiles, whose pipeline fills and drains in fewer SM-cycles per row
+// (measured on B200: the pair kernel is faster from 16384 keys up, the
+// single-CTA one at 8192 and below).
+constexpr int kPairMinKeyTiles = 96;
+std::atomic<int> g_attn_kernel{B2A_ATTN_KERNEL_AUTO};
 
-template <bool PARTIAL>
+bool use_pair(int d, int Skv) {
+  if (d != 128) return false;
+  const int choice = g_attn_kernel.load(std::memory_order_relaxed);
+  if (choice == B2A_ATTN_KERNEL_SINGLE) return false;
+  if (choice == B2A_ATTN_KERNEL_PAIR) return true;
+  return (Skv + 127) / 128 >= kPairMinKeyTiles;
+}
+
+template <int MODE>
 int launch_attn_pair(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int ld_q,
                      int ld_k, int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
   using C = b2a::AttnPairShape;
@@ -188,7 +203,7 @@ int launch_attn_pair(const void* q, const void* k, const void* v, int Sq, int Sk
   prm.Skv = Skv;
   prm.H = H;
   prm.scale_log2 = scale * kLog2e;
-  auto kern = b2a::attn_pair_kernel<PARTIAL>;
+  auto kern = b2a::attn_pair_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   // two CTAs (one cluster) per 256 query rows
@@ -197,6 +212,14 @@ int launch_attn_pair(const void* q, const void* k, const void* v, int Sq, int Sk
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return B2A_OK;
+}
+
+template <int MODE>
+int launch_any(const void* q, const void* k, const void* v, int Sq, int Skv, int H, int d, int ld_q, int ld_k,
+               int ld_v, float scale, b2a::AttnParams prm, cudaStream_t stream) {
+  if (use_pair(d, Skv)) return launch_attn_pair<MODE>(q, k, v, Sq, Skv, H, ld_q, ld_k, ld_v, scale, prm, stream);
+  if (d == 128) return launch_attn<128, MODE>(q, k, v, Sq, Skv, H, ld_q, ld_k, ld_v, scale, prm, stream);
+  return launch_attn<64, MODE>(q, k, v, Sq, Skv, H, ld_q, ld_k, ld_v, scale, prm, stream);
 }
 
 int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
@@ -213,8 +236,7 @@ int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   prm.ld_o = ld_o;
   prm.lse = lse;
   prm.status = di->status;
-  if (d == 128) return launch_attn_pair<false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
-  return launch_attn<64, false>(q, k, v, S, S, H, ld_q, ld_k, ld_v, scale, prm, stream);
+  return launch_any<b2a::kModeFwd>(q, k, v, S, S, H, d, ld_q, ld_k, ld_v, scale, prm, stream);
 }
 
 int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_part,
@@ -237,8 +259,32 @@ int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, f
   prm.o_part = o_part;
   prm.lse_part = lse_part;
   prm.status = di->status;
-  if (d == 128) return launch_attn_pair<true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
-  return launch_attn<64, true>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
+  return launch_any<b2a::kModePartial>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
+}
+
+int attn_accum_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_acc, float* lse_acc,
+                    uint16_t* out, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_kv,
+                    cudaStream_t stream) {
+  int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_kv, ld_kv);
+  if (st != B2A_OK) return st;
+  if (!o_acc || !lse_acc || !aligned16(o_acc) || (reinterpret_cast<uintptr_t>(lse_acc) & 3u))
+    return B2A_ERR_INVALID_ARG;
+  if (out && !aligned16(out)) return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  if (Skv == 0) {
+    if (!out) return B2A_OK;
+    b2a::attn_accum_empty_kernel<<<di->sm_count * 4, 256, 0, stream>>>(o_acc, lse_acc, out, Sq, H, d);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+  }
+  b2a::AttnParams prm{};
+  prm.o_part = o_acc;
+  prm.lse_part = lse_acc;
+  prm.out = out;
+  prm.ld_o = H * d;
+  prm.status = di->status;
+  return launch_any<b2a::kModeAccum>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
 }
 
 int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
@@ -377,6 +423,22 @@ int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const uint16_t*
                            static_cast<cudaStream_t>(stream));
 }
 
+int attn_fwd_accumulate(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk, float* o_acc,
+                        float* lse_acc, uint16_t* out, int Sq, int Skv, int H, int d, float scale, int ld_q,
+                        int ld_kv, void* stream) {
+  return attn_accum_impl(q, k_chunk, v_chunk, o_acc, lse_acc, out, Sq, Skv, H, d, scale, ld_q, ld_kv,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int b2a_set_attn_kernel(int choice) {
+  if (choice != B2A_ATTN_KERNEL_AUTO && choice != B2A_ATTN_KERNEL_SINGLE && choice != B2A_ATTN_KERNEL_PAIR)
+    return B2A_ERR_INVALID_ARG;
+  g_attn_kernel.store(choice, std::memory_order_relaxed);
+  return B2A_OK;
+}
+
+int b2a_get_attn_kernel(void) { return g_attn_kernel.load(std::memory_order_relaxed); }
+
 int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S,
                int H, int d, void* stream) {
   return attn_merge_impl(o_parts, lse_parts, P, out, lse_out, S, H, d, static_cast<cudaStream_t>(stream));
@@ -507,7 +569,7 @@ const char* b2a_status_string(int status) {
 
 int b2a_last_cuda_error(void) { return t_last_cuda_error; }
 
-int b2a_version(void) { return 100; }
+int b2a_version(void) { return 101; }
 
 #ifdef B2A_TRACE
 // Trace builds only: choose the traced CTA, then read the event table

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.b2a_version() == 100
+    assert lib.b2a_version() == 101
     assert lib.b2a_status_string(0) == b"ok"
     assert lib.b2a_status_string(1) == b"invalid argument"
     assert lib.b2a_status_string(4) == b"device-side wait timed out"
@@ -81,6 +81,37 @@ def test_partial_and_merge_reject(lib):
     assert m(FAKE, FAKE, 2, FAKE, None, 16, 2, 80, None) == 1     # d
     assert m(FAKE + 4, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1  # alignment
     assert m(None, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1
+
+
+def test_accumulate_rejects(lib):
+    a = lib.attn_fwd_accumulate
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 4, 2, 64, 0.1, 128, 128, None)
+
+    def call(**kw):
+        names = ["q", "k", "v", "o", "lse", "out", "Sq", "Skv", "H", "d", "scale", "ld_q", "ld_kv", "s"]
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return a(*[args[n] for n in names])
+    assert call(o=None) == 1
+    assert call(lse=None) == 1
+    assert call(o=FAKE + 4) == 1
+    assert call(lse=FAKE + 2) == 1
+    assert call(out=FAKE + 2) == 1
+    assert call(Sq=0) == 1
+    assert call(Skv=-1) == 1
+    assert call(d=96) == 1
+    assert call(scale=0.0) == 1
+    assert call(ld_kv=100) == 1
+
+
+def test_attn_kernel_choice(lib):
+    assert lib.b2a_get_attn_kernel() == 0
+    for c in (1, 2, 0):
+        assert lib.b2a_set_attn_kernel(c) == 0
+        assert lib.b2a_get_attn_kernel() == c
+    assert lib.b2a_set_attn_kernel(3) == 1
+    assert lib.b2a_set_attn_kernel(-1) == 1
+    assert lib.b2a_get_attn_kernel() == 0
 
 
 def test_gemm_rejects(lib):
