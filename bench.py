@@ -50,7 +50,12 @@ def parse():
                     help="override the workload's number of KV chunks P")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--attn-kernel", default="auto", choices=["auto", "single", "pair"],
+                    help="head-dim-128 attention kernel (default: chosen by key count)")
     return ap.parse_args()
+
+
+ATTN_KERNEL_CHOICE = {"auto": 0, "single": 1, "pair": 2}
 
 
 # ------------------------------------------------------------ distributed --
@@ -172,9 +177,11 @@ def peaks():
             "source": "fallback (profiling recipe figures)"}
 
 
-def attn_kernel_name(d: int) -> str:
-    """The monolithic attention kernel the library launches for head dim ``d``."""
-    return "attn_pair_kernel<false>" if d == 128 else f"attn_fwd_kernel<{d},false>"
+def attn_kernel_name(b2a, d: int, Skv: int) -> str:
+    """The monolithic attention kernel the library launches for these sizes."""
+    if b2a.attn_kernel_for(d, Skv) == b2a.ATTN_KERNEL_PAIR:
+        return "attn_pair_kernel<0>"
+    return f"attn_fwd_kernel<{d}, 0, 0>"
 
 
 def committed_traffic(kernel: str, workload: str):
@@ -236,6 +243,7 @@ def run_ours(args, rank, world, local):
     import long_context_bidirectional_b200 as b2a
 
     w = W.ATTN_WORKLOADS[args.workload]
+    b2a.set_attn_kernel(ATTN_KERNEL_CHOICE[args.attn_kernel])
     P = max(args.chunks or w.P, 1)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -335,6 +343,33 @@ def run_ours(args, rank, world, local):
     ring_ms = reduce_max(ra.elapsed_time(rb) / n_ring, world)
     del o_acc, lse_acc, out_r
 
+    # Per-rank shapes of the context-parallel variants (8 ranks), on this GPU:
+    # AllGather-KV rank 3 (its 1/8 of the query rows against every key) and
+    # Ulysses rank 3 (every row for 1/8 of the heads).  Not part of ``value``.
+    def time_calls(fn, n=5):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        b2a.check_status(stream)
+        return reduce_max(a.elapsed_time(b) / n, world)
+
+    lo, hi = b2a.chunk_bounds(S, 8)[3]
+    cp_out = torch.empty((hi - lo, H, d), dtype=torch.float16, device=dev)
+    ag_ms = time_calls(lambda: b2a.attn_fwd_gathered_kv(qd[lo:hi], kd, vd, out=cp_out, return_lse=False,
+                                                        scale=w.scale, stream=stream))
+    hs = slice(3 * (H // 8), 4 * (H // 8)) if H >= 8 else slice(0, H)
+    nh = hs.stop - hs.start
+    uly_ms = time_calls(lambda: b2a.attn_fwd(qd[:, hs], kd[:, hs], vd[:, hs], out=out[:, hs], return_lse=False,
+                                             scale=w.scale, stream=stream))
+    del cp_out
+
     # end to end from pinned host memory through the C-ABI host entry point
     e2e = None
     if not args.no_e2e:
@@ -375,7 +410,7 @@ def run_ours(args, rank, world, local):
         cpu = cpu_baseline(w)
 
     clocks = clk.summary()
-    traffic = committed_traffic("attn_fwd", w.name)
+    traffic = committed_traffic(attn_kernel_name(b2a, d, S), w.name)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -383,11 +418,11 @@ def run_ours(args, rank, world, local):
         "config": {"workload": w.name, "S": S, "H": H, "d": d, "P": P, "batch": 1,
                    "q_sigma": w.q_sigma, "kv_sigma": w.kv_sigma,
                    "step": f"attn_fwd + {P} x attn_fwd_partial + attn_merge",
-                   "step_flops": step_flops,
+                   "step_flops": step_flops, "attn_kernel": args.attn_kernel,
                    "l2": f"inputs larger than L2 (Q,K,V {3 * S * H * d * 2 / 2**20:.0f} MiB, "
                          f"partials {P * S * H * d * 4 / 2**20:.0f} MiB per step)",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(d),
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(b2a, d, S),
                      "achieved": mono_tflops, "peak": pk["tc_burst"], "unit": "TFLOP/s",
                      "frac": mono_tflops / pk["tc_burst"],
                      "frac_of_sustained_peak": mono_tflops / pk["tc_sustained"],
@@ -402,6 +437,12 @@ def run_ours(args, rank, world, local):
                     "ring_pass_ms": ring_ms,
                     "ring_pass_tflops": w.flops / (ring_ms * 1e-3) / 1e12,
                     "ring_pass": f"{P} x attn_fwd_accumulate in place (not in value)",
+                    "cp_gather_kv_rank_ms": ag_ms,
+                    "cp_gather_kv_rank_tflops": 4.0 * (hi - lo) * S * d * H / (ag_ms * 1e-3) / 1e12,
+                    "cp_ulysses_rank_ms": uly_ms,
+                    "cp_ulysses_rank_tflops": 4.0 * S * S * d * nh / (uly_ms * 1e-3) / 1e12,
+                    "cp_ranks": f"8-way: AllGather-KV rank 3 ({hi - lo} rows x {S} keys), Ulysses rank 3 "
+                                f"({nh} of {H} heads); not in value",
                     "merge_hbm_frac": merge_gbs / pk["hbm_gbs"], "merge_bytes": merge_bytes},
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -422,6 +463,7 @@ def run_stack(args, rank, world, local):
     import long_context_bidirectional_b200 as b2a
 
     w = W.STACK_WORKLOADS[args.workload]
+    b2a.set_attn_kernel(ATTN_KERNEL_CHOICE[args.attn_kernel])
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     S, H, d, h = w.S, w.H, w.d, w.hidden
@@ -488,7 +530,7 @@ def run_stack(args, rank, world, local):
         "kernels": {"qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms * 1e-3) / 1e12,
                     "attn_fwd_ms": att_ms, "attn_fwd_tflops": f_att / (att_ms * 1e-3) / 1e12,
                     "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms * 1e-3) / 1e12},
-        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(d),
+        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(b2a, d, S),
                      "achieved": f_att / (att_ms * 1e-3) / 1e12, "peak": pk["tc_burst"], "unit": "TFLOP/s",
                      "frac": f_att / (att_ms * 1e-3) / 1e12 / pk["tc_burst"], "peak_source": pk["source"],
                      "traffic": None, "algorithmic": "4*S^2*d*H flops per launch"},

@@ -73,6 +73,41 @@ B2A_API int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
              int S, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o, void* stream);
 
 /*
+ * attn_fwd_batched -- attn_fwd over a batch in the pages' (S, B, hidden)
+ * activation layout ("Multi-Device Attention Inference with TensorRT",
+ * Generating the ONNX Models: input/output (sequence_length, batch_size,
+ * 4096)).  Batch b is the strided view that starts at column b*H*d with row
+ * stride B*H*d; the call runs attn_fwd on each batch in turn on `stream`.
+ *
+ * q, k, v, out  device fp16 [S, B, H, d] contiguous.
+ * lse           device fp32 [B, H, S], or NULL.
+ * B >= 1 and B*H*d <= 2^31 - 1; other requirements as attn_fwd.
+ */
+B2A_API int attn_fwd_batched(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                             float* lse, int S, int B, int H, int d, float scale, void* stream);
+
+/*
+ * attn_fwd_gathered_kv -- attn_fwd for Sq query rows against Skv keys: the
+ * attention one rank computes in the AllGather-KV form of context
+ * parallelism, where each rank keeps its own chunk of query rows and
+ * gathers K and V from all ranks before attention (TensorRT 11.0
+ * multi-device article, the three context-parallel implementations,
+ * AllGather-KV; the sample's sharding hint gathers K/V and keeps Q local:
+ * "Multi-Device Attention Inference with TensorRT", What is hint.json?).
+ *   out[i, h, :] = sum_j softmax_j(scale * q[i,h,:] . k[j,h,:]) * v[j, h, :]
+ *   lse[h, i]    = ln sum_j exp(scale * q[i,h,:] . k[j,h,:])
+ *
+ * q    device fp16 [Sq, H, d], row stride ld_q.
+ * k, v device fp16 [Skv, H, d], row strides ld_k, ld_v.
+ * out  device fp16 [Sq, H, d], row stride ld_o;  lse fp32 [H, Sq] or NULL.
+ * Sq >= 1, Skv >= 1; other requirements as attn_fwd (attn_fwd is the case
+ * Sq = Skv = S).
+ */
+B2A_API int attn_fwd_gathered_kv(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                                 float* lse, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_k,
+                                 int ld_v, int ld_o, void* stream);
+
+/*
  * attn_fwd_partial -- attention of all queries against one contiguous chunk
  * of keys, the per-step work of ring attention (TensorRT 11.0 multi-device
  * article, the three context-parallel implementations, Ring Attention).
@@ -278,6 +313,9 @@ B2A_API int b2a_last_cuda_error(void);
 enum { B2A_ATTN_KERNEL_AUTO = 0, B2A_ATTN_KERNEL_SINGLE = 1, B2A_ATTN_KERNEL_PAIR = 2 };
 B2A_API int b2a_set_attn_kernel(int choice);
 B2A_API int b2a_get_attn_kernel(void);
+/* The kernel a call with head dim d and Skv keys would use now:
+   B2A_ATTN_KERNEL_SINGLE or B2A_ATTN_KERNEL_PAIR. */
+B2A_API int b2a_attn_kernel_for(int d, int Skv);
 
 /* Library ABI version (major*100 + minor). */
 B2A_API int b2a_version(void);

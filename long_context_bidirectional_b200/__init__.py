@@ -22,9 +22,9 @@ import torch
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libb200attn.so")
 
 __all__ = [
-    "B2AError", "lib", "attn_fwd", "attn_fwd_partial", "attn_fwd_accumulate", "attn_merge", "attn_chunked",
-    "attn_ring", "set_attn_kernel", "get_attn_kernel", "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE",
-    "ATTN_KERNEL_PAIR",
+    "B2AError", "lib", "attn_fwd", "attn_fwd_batched", "attn_fwd_gathered_kv", "attn_fwd_partial", "attn_fwd_accumulate",
+    "attn_merge", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
+    "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PAIR",
     "qkv_proj", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
     "host_workspace_bytes", "check_status",
     "chunk_bounds", "library_path",
@@ -40,10 +40,13 @@ _f = ctypes.c_float
 
 _SIGS = {
     "attn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _i, _i, _i, _vp]),
+    "attn_fwd_batched": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]),
+    "attn_fwd_gathered_kv": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _i, _vp]),
     "attn_fwd_partial": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_fwd_accumulate": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "b2a_set_attn_kernel": (_i, [_i]),
     "b2a_get_attn_kernel": (_i, []),
+    "b2a_attn_kernel_for": (_i, [_i, _i]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
@@ -157,6 +160,46 @@ def attn_fwd(q, k, v, out=None, lse=None, scale=None, return_lse=True, stream=No
     return out, lse
 
 
+def attn_fwd_batched(q, k, v, out=None, lse=None, scale=None, return_lse=True, stream=None):
+    """attn_fwd over ``[S, B, H, d]`` contiguous tensors (the (S, B, hidden)
+    layout); returns ``(out [S,B,H,d], lse [B,H,S])``."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.float16):
+            raise TypeError(f"{name} must be a float16 CUDA tensor")
+        if t.dim() != 4 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{name} must be contiguous [S, B, H, d] like q")
+    S, B, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if not (out.is_contiguous() and out.shape == q.shape and out.dtype == torch.float16):
+        raise ValueError("out must be contiguous float16 [S, B, H, d]")
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _call("attn_fwd_batched", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+          S, B, H, d, _default_scale(d, scale), _stream(stream))
+    return out, lse
+
+
+def attn_fwd_gathered_kv(q, k, v, out=None, lse=None, scale=None, return_lse=True, stream=None):
+    """One AllGather-KV context-parallel rank: its ``q [Sq,H,d]`` rows against
+    all ``k, v [Skv,H,d]``; returns ``(out [Sq,H,d] fp16, lse [H,Sq])``."""
+    Sq, H, d = q.shape
+    ld_q = _check_qkv("q", q)
+    ld_k = _check_qkv("k", k, H, d)
+    ld_v = _check_qkv("v", v, H, d)
+    Skv = k.shape[0]
+    if v.shape[0] != Skv:
+        raise ValueError("k and v need the same length")
+    if out is None:
+        out = torch.empty((Sq, H, d), dtype=torch.float16, device=q.device)
+    ld_o = _check_qkv("out", out, H, d)
+    if lse is None and return_lse:
+        lse = torch.empty((H, Sq), dtype=torch.float32, device=q.device)
+    _call("attn_fwd_gathered_kv", q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+          Sq, Skv, H, d, _default_scale(d, scale), ld_q, ld_k, ld_v, ld_o, _stream(stream))
+    return out, lse
+
+
 def attn_fwd_partial(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None, stream=None):
     """Attention of all queries against one key chunk; returns ``(o_part, lse_part)``."""
     Sq, H, d = q.shape
@@ -239,6 +282,11 @@ def set_attn_kernel(choice: int) -> None:
 
 def get_attn_kernel() -> int:
     return int(_get_lib().b2a_get_attn_kernel())
+
+
+def attn_kernel_for(d: int, Skv: int) -> int:
+    """ATTN_KERNEL_SINGLE or ATTN_KERNEL_PAIR: what a call with these sizes uses now."""
+    return int(_get_lib().b2a_attn_kernel_for(int(d), int(Skv)))
 
 
 def attn_merge(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stream=None):

@@ -223,9 +223,10 @@ int launch_any(const void* q, const void* k, const void* v, int Sq, int Skv, int
 }
 
 int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
-                  int S, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
+                  int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
                   cudaStream_t stream) {
-  int st = validate_attn(q, k, v, S, S, H, d, scale, ld_q, ld_k, ld_v);
+  if (Skv < 1) return B2A_ERR_INVALID_ARG;
+  int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_k, ld_v);
   if (st != B2A_OK) return st;
   if (!out || !aligned16(out) || !good_ld(ld_o, H, d)) return B2A_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return B2A_ERR_INVALID_ARG;
@@ -236,7 +237,7 @@ int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   prm.ld_o = ld_o;
   prm.lse = lse;
   prm.status = di->status;
-  return launch_any<b2a::kModeFwd>(q, k, v, S, S, H, d, ld_q, ld_k, ld_v, scale, prm, stream);
+  return launch_any<b2a::kModeFwd>(q, k, v, Sq, Skv, H, d, ld_q, ld_k, ld_v, scale, prm, stream);
 }
 
 int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_part,
@@ -412,7 +413,31 @@ extern "C" {
 
 int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse, int S,
              int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o, void* stream) {
-  return attn_fwd_impl(q, k, v, out, lse, S, H, d, scale, ld_q, ld_k, ld_v, ld_o,
+  return attn_fwd_impl(q, k, v, out, lse, S, S, H, d, scale, ld_q, ld_k, ld_v, ld_o,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_batched(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse, int S,
+                     int B, int H, int d, float scale, void* stream) {
+  if (B < 1 || H < 1 || S < 1) return B2A_ERR_INVALID_ARG;
+  const long long row = static_cast<long long>(B) * H * d;
+  if (row > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const int ld = static_cast<int>(row);
+  const size_t hd = static_cast<size_t>(H) * d;
+  for (int b = 0; b < B; ++b) {
+    const size_t off = static_cast<size_t>(b) * hd;
+    float* lse_b = lse ? lse + static_cast<size_t>(b) * H * S : nullptr;
+    const int st = attn_fwd_impl(q + off, k + off, v + off, out + off, lse_b, S, S, H, d, scale, ld, ld, ld, ld,
+                                 static_cast<cudaStream_t>(stream));
+    if (st != B2A_OK) return st;
+  }
+  return B2A_OK;
+}
+
+int attn_fwd_gathered_kv(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
+                         int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
+                         void* stream) {
+  return attn_fwd_impl(q, k, v, out, lse, Sq, Skv, H, d, scale, ld_q, ld_k, ld_v, ld_o,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -439,6 +464,8 @@ int b2a_set_attn_kernel(int choice) {
 
 int b2a_get_attn_kernel(void) { return g_attn_kernel.load(std::memory_order_relaxed); }
 
+int b2a_attn_kernel_for(int d, int Skv) { return use_pair(d, Skv) ? B2A_ATTN_KERNEL_PAIR : B2A_ATTN_KERNEL_SINGLE; }
+
 int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S,
                int H, int d, void* stream) {
   return attn_merge_impl(o_parts, lse_parts, P, out, lse_out, S, H, d, static_cast<cudaStream_t>(stream));
@@ -463,8 +490,8 @@ int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   int st = gemm_impl(x, w_qkv, nullptr, qkv_ws, S, 3 * hi, hi, stream);
   if (st != B2A_OK) return st;
-  st = attn_fwd_impl(qkv_ws, qkv_ws + h, qkv_ws + 2 * h, attn_ws, nullptr, S, H, d, scale, 3 * hi, 3 * hi,
-                     3 * hi, hi, stream);
+  st = attn_fwd_impl(qkv_ws, qkv_ws + h, qkv_ws + 2 * h, attn_ws, nullptr, S, S, H, d, scale, 3 * hi,
+                     3 * hi, 3 * hi, hi, stream);
   if (st != B2A_OK) return st;
   return gemm_impl(attn_ws, w_o, x, y, S, hi, hi, stream);
 }
@@ -518,7 +545,7 @@ int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   if ((e = cudaMemcpyAsync(dv, v, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
   const int ld = H * d;
   if (P == 1) {
-    st = attn_fwd_impl(dq, dk, dv, dout, dlse, S, H, d, scale, ld, ld, ld, ld, stream);
+    st = attn_fwd_impl(dq, dk, dv, dout, dlse, S, S, H, d, scale, ld, ld, ld, ld, stream);
   } else {
     float* op = reinterpret_cast<float*>(ws + w.o_parts);
     float* lp = reinterpret_cast<float*>(ws + w.lse_parts);

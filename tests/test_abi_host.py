@@ -104,6 +104,19 @@ def test_accumulate_rejects(lib):
     assert call(ld_kv=100) == 1
 
 
+def test_gathered_kv_and_batched_reject(lib):
+    g = lib.attn_fwd_gathered_kv
+    assert g(FAKE, FAKE, FAKE, FAKE, None, 4, 0, 2, 64, 0.1, 128, 128, 128, 128, None) == 1   # Skv = 0
+    assert g(FAKE, FAKE, FAKE, FAKE, None, 0, 4, 2, 64, 0.1, 128, 128, 128, 128, None) == 1   # Sq = 0
+    assert g(FAKE, FAKE, FAKE, FAKE, None, 4, 4, 2, 96, 0.1, 128, 128, 128, 128, None) == 1   # d
+    assert g(FAKE, FAKE, FAKE, None, None, 4, 4, 2, 64, 0.1, 128, 128, 128, 128, None) == 1   # out
+    b = lib.attn_fwd_batched
+    assert b(FAKE, FAKE, FAKE, FAKE, None, 16, 0, 2, 64, 0.1, None) == 1    # B = 0
+    assert b(FAKE, FAKE, FAKE, FAKE, None, 0, 2, 2, 64, 0.1, None) == 1     # S = 0
+    assert b(FAKE, FAKE, FAKE, FAKE, None, 16, 2, 2, 80, 0.1, None) == 1    # d
+    assert b(FAKE, FAKE, FAKE, FAKE, None, 16, 70000, 256, 128, 0.1, None) == 2  # B*H*d too wide
+
+
 def test_attn_kernel_choice(lib):
     assert lib.b2a_get_attn_kernel() == 0
     for c in (1, 2, 0):

@@ -82,11 +82,14 @@ SEQ8K = AttnWorkload("s8192_h32_d128", S=8192, H=32, d=128, P=2)
 SEQ32K = AttnWorkload("s32768_h32_d128_qsig4", S=32768, H=32, d=128, q_sigma=4.0, P=8)
 SEQ64K = AttnWorkload("s65536_h32_d128", S=65536, H=32, d=128, P=1)
 SEQ8K_H64 = AttnWorkload("s8192_h64_d128", S=8192, H=64, d=128, P=1)
+# The sample's default run ("Multi-Device Attention Inference with TensorRT",
+# Running the Sample: --sequence-length 56320 --batch-size 1).
+SEQ56K = AttnWorkload("s56320_h32_d128", S=56320, H=32, d=128, P=1)
 STACK6 = StackWorkload("stack6_s32768_h4096", S=32768, H=32, d=128, blocks=6)
 # A shorter stack that a full (unsampled) FP64 pass can follow end to end.
 STACK6_S2048 = StackWorkload("stack6_s2048_h4096", S=2048, H=32, d=128, blocks=6)
 
-ATTN_WORKLOADS = {w.name: w for w in (TINY, SEQ8K, SEQ32K, SEQ64K, SEQ8K_H64)}
+ATTN_WORKLOADS = {w.name: w for w in (TINY, SEQ8K, SEQ32K, SEQ64K, SEQ8K_H64, SEQ56K)}
 STACK_WORKLOADS = {w.name: w for w in (STACK6, STACK6_S2048)}
 
 
