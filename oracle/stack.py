@@ -16,7 +16,12 @@ Readings where the pages are silent:
   head-major (column ``head*d + e``).
 * The block output is ``x + Z`` (a residual add).
 * RMSNorm, listed in the sample model without placement or epsilon, is not
-  part of this stack.
+  part of ``block``/``stack``.  ``qkv_qknorm`` gives the reading used when it
+  is asked for: the sample lists "Q/K/V projections, RMSNorm, scaled
+  dot-product attention, output projection" in that order, so the norm acts
+  on the projected q and k, per head, before attention (``qkv_qknorm``
+  below; epsilon 1e-6 unless given, one weight vector of length d for q and
+  one for k, shared by the heads).
 * Tensors are rounded to fp16 (round-to-nearest-even) exactly where the
   library stores fp16: after the QKV projection, after attention, after the
   residual add.  Everything between those boundaries is float64.
@@ -38,11 +43,39 @@ def linear(x, w) -> np.ndarray:
     return np.asarray(x).astype(np.float64) @ np.asarray(w).astype(np.float64).T
 
 
-def block(x16, w_qkv16, w_o16, H: int, d: int, scale: float):
-    """One block on all rows.  Returns ``(y16, qkv16, a16)``, all fp16."""
+def rmsnorm(x, g, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: ``x / sqrt(mean(x**2) + eps) * g``, float64."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)
+
+
+def qkv_qknorm(x16, w_qkv16, g_q16, g_k16, H: int, d: int, eps: float):
+    """The fused QKV projection with the RMSNorm reading applied: every head
+    of q and of k (``d`` features each) is RMS-normalised and scaled by the
+    per-feature weights ``g_q`` / ``g_k`` (length ``d``, shared by the heads),
+    from the exact projection; v is left as projected.  One fp16 rounding.
+    Returns ``qkv16 [S, 3*H*d]``.
+    """
     S = x16.shape[0]
     h = H * d
-    qkv16 = round16(linear(x16, w_qkv16))                  # [S, 3h]
+    acc = linear(x16, w_qkv16)                             # [S, 3h] exact
+    q = rmsnorm(acc[:, 0:h].reshape(S, H, d), g_q16, eps).reshape(S, h)
+    k = rmsnorm(acc[:, h:2 * h].reshape(S, H, d), g_k16, eps).reshape(S, h)
+    return round16(np.concatenate([q, k, acc[:, 2 * h:3 * h]], axis=1))
+
+
+def block(x16, w_qkv16, w_o16, H: int, d: int, scale: float, norm=None):
+    """One block on all rows.  Returns ``(y16, qkv16, a16)``, all fp16.
+
+    ``norm = (g_q16, g_k16, eps)`` applies the q/k RMSNorm reading.
+    """
+    S = x16.shape[0]
+    h = H * d
+    if norm is None:
+        qkv16 = round16(linear(x16, w_qkv16))              # [S, 3h]
+    else:
+        qkv16 = qkv_qknorm(x16, w_qkv16, norm[0], norm[1], H, d, norm[2])
     q = qkv16[:, 0 * h:1 * h].reshape(S, H, d)
     k = qkv16[:, 1 * h:2 * h].reshape(S, H, d)
     v = qkv16[:, 2 * h:3 * h].reshape(S, H, d)

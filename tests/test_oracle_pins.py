@@ -308,6 +308,49 @@ def test_ring_step_order_does_not_matter():
 
 # ----------------------------------------------------------------- stack ----
 
+def test_rmsnorm_closed_forms():
+    # a constant vector c*1: mean square c^2, so with eps = 0 the result is sign(c) * g
+    g = np.array([0.5, -2.0, 3.0, 1.0])
+    np.testing.assert_allclose(ST.rmsnorm(np.full(4, -3.0), g, 0.0), -g, atol=1e-15)
+    # (3, 4) has mean square 12.5: y = (3, 4) / sqrt(12.5 + eps)
+    y = ST.rmsnorm(np.array([3.0, 4.0]), np.ones(2), 0.5)
+    np.testing.assert_allclose(y, np.array([3.0, 4.0]) / math.sqrt(13.0), atol=1e-15)
+    # with eps = 0 and g = 1 every normalised vector has mean square 1,
+    # and scaling the input by c > 0 changes nothing
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((5, 7, 16)) * 3
+    yn = ST.rmsnorm(x, np.ones(16), 0.0)
+    np.testing.assert_allclose(np.mean(yn * yn, axis=-1), 1.0, atol=1e-13)
+    np.testing.assert_allclose(ST.rmsnorm(4.5 * x, np.ones(16), 0.0), yn, atol=1e-13)
+    # eps shrinks the mean square to ms / (ms + eps)
+    ms = np.mean(x * x, axis=-1)
+    ye = ST.rmsnorm(x, np.ones(16), 0.25)
+    np.testing.assert_allclose(np.mean(ye * ye, axis=-1), ms / (ms + 0.25), atol=1e-13)
+
+
+def test_qkv_qknorm_against_python_loops():
+    rng = np.random.default_rng(25)
+    S, H, d, K = 3, 2, 4, 5
+    x = rng.standard_normal((S, K)).astype(np.float16)
+    w = rng.standard_normal((3 * H * d, K)).astype(np.float16)
+    gq = rng.standard_normal(d).astype(np.float16)
+    gk = rng.standard_normal(d).astype(np.float16)
+    eps = 1e-3
+    got = ST.qkv_qknorm(x, w, gq, gk, H, d, eps)
+    h = H * d
+    for s in range(S):
+        row = [sum(float(x[s, c]) * float(w[n, c]) for c in range(K)) for n in range(3 * h)]
+        for sec, g in ((0, gq), (1, gk)):
+            for hh in range(H):
+                seg = row[sec * h + hh * d: sec * h + (hh + 1) * d]
+                r = math.sqrt(sum(t * t for t in seg) / d + eps)
+                for e in range(d):
+                    want = np.float16(seg[e] / r * float(g[e]))
+                    assert got[s, sec * h + hh * d + e] == want
+        for n in range(2 * h, 3 * h):   # v is left as projected
+            assert got[s, n] == np.float16(row[n])
+
+
 def test_round16_matches_ieee_half_from_struct():
     vals = [0.1, 1 / 3, 2049.0, 2051.0, 65504.0, -7.123456, 1e-5, 3.0e-8, 1.0 + 2 ** -11]
     got = ST.round16(np.array(vals))
