@@ -191,6 +191,30 @@ B2A_API int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, in
              void* stream);
 
 /*
+ * qkv_proj_qknorm -- qkv_proj with the block's RMSNorm applied to q and k.
+ *
+ * The sample's block lists "Q/K/V projections, RMSNorm, scaled dot-product
+ * attention, output projection" ("Multi-Device Attention Inference with
+ * TensorRT", Generating the ONNX Models) without placement or epsilon; the
+ * reading taken here normalises every head of q and of k after the
+ * projection, in the GEMM's epilogue from the fp32 accumulator:
+ *   q[i, h, :] <- q[i, h, :] / sqrt(mean_e q[i, h, e]^2 + eps) * g_q
+ *   k[i, h, :] <- k[i, h, :] / sqrt(mean_e k[i, h, e]^2 + eps) * g_k
+ * v is stored as projected; each value is rounded once to fp16.
+ *
+ * x      device fp16 [M, K];  w_qkv device fp16 [3*H*d, K] ([out, in]).
+ * g_q,
+ * g_k    device fp16 [d] per-feature weights (shared by the heads), 16-byte
+ *        aligned.
+ * qkv    device fp16 [M, 3*H*d] (columns [q | k | v], head-major).
+ * d in {64, 128}, H >= 1, eps >= 0 and finite (1e-6 is the usual choice);
+ * other requirements as qkv_proj.
+ */
+B2A_API int qkv_proj_qknorm(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* g_q,
+                            const uint16_t* g_k, uint16_t* qkv, int M, int H, int d, int K, float eps,
+                            void* stream);
+
+/*
  * out_proj -- output projection with residual, y = residual + a * w_o^T
  * (section 3, step 4 of the same lesson: Z = Concat(heads) W_O; the block
  * adds its input back).  The residual is added to the fp32 accumulator and
@@ -227,6 +251,15 @@ B2A_API int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* res
 B2A_API int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o, uint16_t* y,
                            uint16_t* qkv_ws, uint16_t* attn_ws, int S, int H, int d, float scale,
                            void* stream);
+
+/*
+ * attn_block_fwd_qknorm -- attn_block_fwd with qkv_proj_qknorm as its first
+ * step (g_q, g_k, eps as there; both NULL: exactly attn_block_fwd).
+ */
+B2A_API int attn_block_fwd_qknorm(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* g_q,
+                                  const uint16_t* g_k, float eps, const uint16_t* w_o, uint16_t* y,
+                                  uint16_t* qkv_ws, uint16_t* attn_ws, int S, int H, int d, float scale,
+                                  void* stream);
 
 /*
  * attn_block_fwd_static -- attn_block_fwd for callers that cannot allocate.

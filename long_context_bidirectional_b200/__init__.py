@@ -25,7 +25,7 @@ __all__ = [
     "B2AError", "lib", "attn_fwd", "attn_fwd_batched", "attn_fwd_gathered_kv", "attn_fwd_partial", "attn_fwd_accumulate",
     "attn_merge", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
     "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PAIR",
-    "qkv_proj", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
+    "qkv_proj", "qkv_proj_qknorm", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
     "host_workspace_bytes", "check_status",
     "chunk_bounds", "library_path",
 ]
@@ -52,6 +52,8 @@ _SIGS = {
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "attn_block_fwd_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "out_proj": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp]),
+    "qkv_proj_qknorm": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]),
+    "attn_block_fwd_qknorm": (_i, [_vp, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, ctypes.c_uint64, _vp]),
     "attn_fwd_host_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),
     "b2a_check_status": (_i, [_vp]),
@@ -353,6 +355,25 @@ def qkv_proj(x, w_qkv, out=None, stream=None):
     return out
 
 
+def qkv_proj_qknorm(x, w_qkv, g_q, g_k, H: int, d: int, eps: float = 1e-6, out=None, stream=None):
+    """``out = x @ w_qkv.T`` with every q and k head RMS-normalised and scaled
+    by ``g_q`` / ``g_k`` ([d] fp16) in the GEMM epilogue; v as projected."""
+    M, K = x.shape
+    N = 3 * H * d
+    _check_mat("x", x)
+    _check_mat("w_qkv", w_qkv, N, K)
+    for name, g in (("g_q", g_q), ("g_k", g_k)):
+        if not (isinstance(g, torch.Tensor) and g.is_cuda and g.dtype == torch.float16
+                and g.is_contiguous() and g.numel() == d):
+            raise ValueError(f"{name} must be a contiguous float16 CUDA tensor of {d} elements")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _check_mat("out", out, M, N)
+    _call("qkv_proj_qknorm", x.data_ptr(), w_qkv.data_ptr(), g_q.data_ptr(), g_k.data_ptr(), out.data_ptr(),
+          M, H, d, K, float(eps), _stream(stream))
+    return out
+
+
 def out_proj(a, w_o, residual=None, out=None, stream=None):
     """``out = residual + a @ w_o.T`` (residual optional, may be ``out``)."""
     M, K = a.shape
@@ -370,8 +391,12 @@ def out_proj(a, w_o, residual=None, out=None, stream=None):
 
 
 def attn_block_fwd(x, w_qkv, w_o, H: int, d: int, out=None, qkv_ws=None, attn_ws=None, scale=None,
-                   stream=None):
-    """One block: ``out = x + attention(split(x @ w_qkv.T)) @ w_o.T``; ``out`` may be ``x``."""
+                   stream=None, qknorm=None):
+    """One block: ``out = x + attention(split(x @ w_qkv.T)) @ w_o.T``; ``out`` may be ``x``.
+
+    ``qknorm = (g_q, g_k, eps)`` runs the projection with the q/k RMSNorm
+    (``attn_block_fwd_qknorm``).
+    """
     S, h = x.shape
     if h != H * d:
         raise ValueError(f"x has {h} columns, expected H*d = {H * d}")
@@ -387,8 +412,18 @@ def attn_block_fwd(x, w_qkv, w_o, H: int, d: int, out=None, qkv_ws=None, attn_ws
         attn_ws = torch.empty((S, h), dtype=torch.float16, device=x.device)
     _check_mat("qkv_ws", qkv_ws, S, 3 * h)
     _check_mat("attn_ws", attn_ws, S, h)
-    _call("attn_block_fwd", x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), out.data_ptr(),
-          qkv_ws.data_ptr(), attn_ws.data_ptr(), S, H, d, _default_scale(d, scale), _stream(stream))
+    if qknorm is None:
+        _call("attn_block_fwd", x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), out.data_ptr(),
+              qkv_ws.data_ptr(), attn_ws.data_ptr(), S, H, d, _default_scale(d, scale), _stream(stream))
+        return out
+    g_q, g_k, eps = qknorm
+    for name, g in (("g_q", g_q), ("g_k", g_k)):
+        if not (isinstance(g, torch.Tensor) and g.is_cuda and g.dtype == torch.float16
+                and g.is_contiguous() and g.numel() == d):
+            raise ValueError(f"{name} must be a contiguous float16 CUDA tensor of {d} elements")
+    _call("attn_block_fwd_qknorm", x.data_ptr(), w_qkv.data_ptr(), g_q.data_ptr(), g_k.data_ptr(), float(eps),
+          w_o.data_ptr(), out.data_ptr(), qkv_ws.data_ptr(), attn_ws.data_ptr(), S, H, d,
+          _default_scale(d, scale), _stream(stream))
     return out
 
 

@@ -319,8 +319,16 @@ int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
 }
 
+// q/k RMSNorm epilogue parameters (null: plain projection).
+struct QkNorm {
+  const uint16_t* g_q;
+  const uint16_t* g_k;
+  int H, d;
+  float eps;
+};
+
 int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t* c, int M, int N, int K,
-              cudaStream_t stream) {
+              cudaStream_t stream, const QkNorm* norm = nullptr) {
   if (!a || !w || !c) return B2A_ERR_INVALID_ARG;
   if (!aligned16(a) || !aligned16(w) || !aligned16(c) || (r && !aligned16(r))) return B2A_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || (N % 8) != 0 || (K % 8) != 0) return B2A_ERR_INVALID_ARG;
@@ -344,13 +352,30 @@ int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t*
   prm.c = c;
   prm.r = r;
   prm.status = di->status;
-  cudaError_t e = cudaFuncSetAttribute(b2a::gemm_tn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       G::SMEM_BYTES);
+  if (norm) {
+    prm.g_q = norm->g_q;
+    prm.g_k = norm->g_k;
+    prm.hsec = norm->H * norm->d;
+    prm.dh = norm->d;
+    prm.eps = norm->eps;
+  }
+  auto kern = norm ? b2a::gemm_tn_kernel<true> : b2a::gemm_tn_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = prm.num_tiles < di->sm_count ? prm.num_tiles : di->sm_count;
-  b2a::gemm_tn_kernel<<<grid, G::THREADS, G::SMEM_BYTES, stream>>>(ta, tb, prm);
+  kern<<<grid, G::THREADS, G::SMEM_BYTES, stream>>>(ta, tb, prm);
   e = cudaGetLastError();
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+
+int qkv_qknorm_impl(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* g_q, const uint16_t* g_k,
+                    uint16_t* qkv, int M, int H, int d, int K, float eps, cudaStream_t stream) {
+  if (!g_q || !g_k || !aligned16(g_q) || !aligned16(g_k)) return B2A_ERR_INVALID_ARG;
+  if (H < 1 || (d != 64 && d != 128) || !std::isfinite(eps) || eps < 0.f) return B2A_ERR_INVALID_ARG;
+  const long long n = 3LL * H * d;
+  if (n > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const QkNorm norm{g_q, g_k, H, d, eps};
+  return gemm_impl(x, w_qkv, nullptr, qkv, M, static_cast<int>(n), K, stream, &norm);
 }
 
 // Static scratch of attn_block_fwd_static: qkv [S, 3h] then the attention
@@ -475,6 +500,11 @@ int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, int M, int
   return gemm_impl(x, w_qkv, nullptr, qkv, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
+int qkv_proj_qknorm(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* g_q, const uint16_t* g_k,
+                    uint16_t* qkv, int M, int H, int d, int K, float eps, void* stream) {
+  return qkv_qknorm_impl(x, w_qkv, g_q, g_k, qkv, M, H, d, K, eps, static_cast<cudaStream_t>(stream));
+}
+
 int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* residual, uint16_t* y, int M, int N,
              int K, void* stream) {
   return gemm_impl(a, w_o, residual, y, M, N, K, static_cast<cudaStream_t>(stream));
@@ -482,13 +512,21 @@ int out_proj(const uint16_t* a, const uint16_t* w_o, const uint16_t* residual, u
 
 int attn_block_fwd(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* w_o, uint16_t* y,
                    uint16_t* qkv_ws, uint16_t* attn_ws, int S, int H, int d, float scale, void* stream_) {
+  return attn_block_fwd_qknorm(x, w_qkv, nullptr, nullptr, 0.f, w_o, y, qkv_ws, attn_ws, S, H, d, scale, stream_);
+}
+
+int attn_block_fwd_qknorm(const uint16_t* x, const uint16_t* w_qkv, const uint16_t* g_q, const uint16_t* g_k,
+                          float eps, const uint16_t* w_o, uint16_t* y, uint16_t* qkv_ws, uint16_t* attn_ws, int S,
+                          int H, int d, float scale, void* stream_) {
   if (!x || !w_qkv || !w_o || !y || !qkv_ws || !attn_ws) return B2A_ERR_INVALID_ARG;
   if (S < 1 || H < 1 || (d != 64 && d != 128) || !good_scale(scale)) return B2A_ERR_INVALID_ARG;
+  if ((g_q == nullptr) != (g_k == nullptr)) return B2A_ERR_INVALID_ARG;
   const long long h = static_cast<long long>(H) * d;
   if (3 * h > INT_MAX) return B2A_ERR_UNSUPPORTED;
   const int hi = static_cast<int>(h);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-  int st = gemm_impl(x, w_qkv, nullptr, qkv_ws, S, 3 * hi, hi, stream);
+  int st = g_q ? qkv_qknorm_impl(x, w_qkv, g_q, g_k, qkv_ws, S, H, d, hi, eps, stream)
+               : gemm_impl(x, w_qkv, nullptr, qkv_ws, S, 3 * hi, hi, stream);
   if (st != B2A_OK) return st;
   st = attn_fwd_impl(qkv_ws, qkv_ws + h, qkv_ws + 2 * h, attn_ws, nullptr, S, S, H, d, scale, 3 * hi,
                      3 * hi, 3 * hi, hi, stream);

@@ -6,7 +6,11 @@
 // Z = Concat(heads) W_O; "Multi-Device Attention Inference with TensorRT",
 // Generating the ONNX Models: Q/K/V and output projections), with weights in
 // the [out, in] layout.  fp16 operands, fp32 accumulation in TMEM, one fp16
-// rounding of (acc + residual) in the epilogue.
+// rounding of (acc + residual) in the epilogue.  A second instantiation
+// applies a per-head RMSNorm to the q and k columns of the fused QKV output
+// in the epilogue (the sample block lists Q/K/V projections, then RMSNorm,
+// then attention: "Multi-Device Attention Inference with TensorRT",
+// Generating the ONNX Models).
 //
 // Persistent kernel, one CTA per SM, 128x256 output tiles, K in steps of 64
 // through a 4-stage TMA ring (128-byte swizzle).  Warp roles:
@@ -27,6 +31,13 @@ struct GemmParams {
   uint16_t* c;          // [M, N] fp16
   const uint16_t* r;    // [M, N] fp16 residual (nullable, may alias c)
   unsigned int* status;
+  // q/k RMSNorm epilogue (gemm_tn_kernel<true>): columns [0, hsec) are q and
+  // [hsec, 2*hsec) are k, in heads of dh columns; each head segment of a row
+  // is scaled by rsqrt(mean of its squares + eps) and by g_q / g_k [dh].
+  const uint16_t* g_q;
+  const uint16_t* g_k;
+  int hsec, dh;
+  float eps;
 };
 
 struct GemmShape {
@@ -61,6 +72,7 @@ __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, 
   nb = in / gsize;
 }
 
+template <bool NORM>
 __global__ void __launch_bounds__(192, 1)
     gemm_tn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                    const GemmParams p) {
@@ -178,35 +190,88 @@ __global__ void __launch_bounds__(192, 1)
       const int row = mb * C::BM + quarter * 32 + lane;
       const bool live = row < p.M;
       const uint32_t t_base = tmem + lane_off + buf * C::BN;
-#pragma unroll 1
-      for (int cb = 0; cb < C::BN; cb += 32) {
-        uint32_t v[32];
-        tmem_ld32(t_base + cb, v);
-        tmem_wait_ld(v);
-        const int col0 = nb * C::BN + cb;
-        if (live) {
+      if constexpr (NORM) {
+        // Head segments of dh columns: q and k heads are normalised from the
+        // fp32 accumulator (read twice from TMEM: sum of squares, then scale),
+        // v heads are stored as they are.  Segments never straddle q|k|v.
+        for (int s0 = 0; s0 < C::BN; s0 += p.dh) {
+          const int cseg = nb * C::BN + s0;
+          if (cseg >= p.N) break;
+          const int sec = cseg / p.hsec;
+          float mul = 1.f;
+          if (sec < 2) {
+            float ss = 0.f;
+            for (int cb = 0; cb < p.dh; cb += 32) {
+              uint32_t v[32];
+              tmem_ld32(t_base + s0 + cb, v);
+              tmem_wait_ld(v);
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = col0 + g * 8;
-            if (col < p.N) {
-              const size_t off = static_cast<size_t>(row) * p.N + col;
-              float add[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-              if (p.r) {
-                const uint4 rv = *reinterpret_cast<const uint4*>(p.r + off);
-                const __half2* rh = reinterpret_cast<const __half2*>(&rv);
+              for (int c = 0; c < 32; ++c) ss = fmaf(__uint_as_float(v[c]), __uint_as_float(v[c]), ss);
+            }
+            mul = rsqrtf(ss / static_cast<float>(p.dh) + p.eps);
+          }
+          const uint16_t* g = sec == 0 ? p.g_q : p.g_k;
+          for (int cb = 0; cb < p.dh; cb += 32) {
+            uint32_t v[32];
+            tmem_ld32(t_base + s0 + cb, v);
+            tmem_wait_ld(v);
+            if (!live) continue;
+            float y[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) y[c] = __uint_as_float(v[c]);
+            if (sec < 2) {
+              const uint4* gv = reinterpret_cast<const uint4*>(g + cb);
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                const uint4 gw = gv[q8];
+                const __half2* gh = reinterpret_cast<const __half2*>(&gw);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                  const float2 f = __half22float2(rh[e]);
-                  add[2 * e] = f.x;
-                  add[2 * e + 1] = f.y;
+                  const float2 gf = __half22float2(gh[e]);
+                  y[q8 * 8 + 2 * e] *= mul * gf.x;
+                  y[q8 * 8 + 2 * e + 1] *= mul * gf.y;
                 }
               }
-              uint4 o;
-              o.x = pack_half2(__uint_as_float(v[g * 8 + 0]) + add[0], __uint_as_float(v[g * 8 + 1]) + add[1]);
-              o.y = pack_half2(__uint_as_float(v[g * 8 + 2]) + add[2], __uint_as_float(v[g * 8 + 3]) + add[3]);
-              o.z = pack_half2(__uint_as_float(v[g * 8 + 4]) + add[4], __uint_as_float(v[g * 8 + 5]) + add[5]);
-              o.w = pack_half2(__uint_as_float(v[g * 8 + 6]) + add[6], __uint_as_float(v[g * 8 + 7]) + add[7]);
-              *reinterpret_cast<uint4*>(p.c + off) = o;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.c + static_cast<size_t>(row) * p.N + cseg + cb);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+              dst[q8] = make_uint4(pack_half2(y[q8 * 8], y[q8 * 8 + 1]), pack_half2(y[q8 * 8 + 2], y[q8 * 8 + 3]),
+                                   pack_half2(y[q8 * 8 + 4], y[q8 * 8 + 5]),
+                                   pack_half2(y[q8 * 8 + 6], y[q8 * 8 + 7]));
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int cb = 0; cb < C::BN; cb += 32) {
+          uint32_t v[32];
+          tmem_ld32(t_base + cb, v);
+          tmem_wait_ld(v);
+          const int col0 = nb * C::BN + cb;
+          if (live) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int col = col0 + g * 8;
+              if (col < p.N) {
+                const size_t off = static_cast<size_t>(row) * p.N + col;
+                float add[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                if (p.r) {
+                  const uint4 rv = *reinterpret_cast<const uint4*>(p.r + off);
+                  const __half2* rh = reinterpret_cast<const __half2*>(&rv);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const float2 f = __half22float2(rh[e]);
+                    add[2 * e] = f.x;
+                    add[2 * e + 1] = f.y;
+                  }
+                }
+                uint4 o;
+                o.x = pack_half2(__uint_as_float(v[g * 8 + 0]) + add[0], __uint_as_float(v[g * 8 + 1]) + add[1]);
+                o.y = pack_half2(__uint_as_float(v[g * 8 + 2]) + add[2], __uint_as_float(v[g * 8 + 3]) + add[3]);
+                o.z = pack_half2(__uint_as_float(v[g * 8 + 4]) + add[4], __uint_as_float(v[g * 8 + 5]) + add[5]);
+                o.w = pack_half2(__uint_as_float(v[g * 8 + 6]) + add[6], __uint_as_float(v[g * 8 + 7]) + add[7]);
+                *reinterpret_cast<uint4*>(p.c + off) = o;
+              }
             }
           }
         }

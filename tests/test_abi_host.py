@@ -117,6 +117,21 @@ def test_gathered_kv_and_batched_reject(lib):
     assert b(FAKE, FAKE, FAKE, FAKE, None, 16, 70000, 256, 128, 0.1, None) == 2  # B*H*d too wide
 
 
+def test_qknorm_rejects(lib):
+    f = lib.qkv_proj_qknorm
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 4 + [ctypes.c_float, ctypes.c_void_p]
+    assert f(FAKE, FAKE, None, FAKE, FAKE, 128, 2, 64, 128, 1e-6, None) == 1      # g_q
+    assert f(FAKE, FAKE, FAKE, FAKE + 8, FAKE, 128, 2, 64, 128, 1e-6, None) == 1  # g_k alignment
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, 96, 128, 1e-6, None) == 1      # d
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, 64, 128, -1.0, None) == 1      # eps < 0
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 2, 64, 128, float("nan"), None) == 1
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 128, 0, 64, 128, 1e-6, None) == 1      # H
+    b = lib.attn_block_fwd_qknorm
+    b.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + [ctypes.c_int] * 3 + \
+        [ctypes.c_float, ctypes.c_void_p]
+    assert b(FAKE, FAKE, FAKE, None, 1e-6, FAKE, FAKE, FAKE, FAKE, 16, 2, 64, 0.1, None) == 1  # one g only
+
+
 def test_attn_kernel_choice(lib):
     assert lib.b2a_get_attn_kernel() == 0
     for c in (1, 2, 0):

@@ -78,3 +78,26 @@ def test_block1_s32768_sampled_rows(b2a):
     check(qkv_ws.cpu().numpy()[rows], rqkv, "block 1 qkv (sampled rows)")
     check(attn_ws.cpu().numpy()[rows], ra, "block 1 attention (sampled rows)")
     check(y.cpu().numpy()[rows], ry, "block 1 output (sampled rows)")
+
+
+def test_block_with_qk_rmsnorm(b2a):
+    # one block with the q/k RMSNorm reading against the oracle's block
+    S, H, d = 1000, 2, 128
+    h = H * d
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((S, h), dtype=np.float32).astype(np.float16)
+    w_qkv = (rng.standard_normal((3 * h, h), dtype=np.float32) * 0.05).astype(np.float16)
+    w_o = (rng.standard_normal((h, h), dtype=np.float32) * 0.05).astype(np.float16)
+    g_q = (1.0 + 0.1 * rng.standard_normal(d)).astype(np.float16)
+    g_k = (1.0 + 0.1 * rng.standard_normal(d)).astype(np.float16)
+    eps, scale = 1e-6, 1 / np.sqrt(d)
+    ry, rqkv, ra = OS.block(x, w_qkv, w_o, H, d, scale, norm=(g_q, g_k, eps))
+    qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device="cuda")
+    attn_ws = torch.empty((S, h), dtype=torch.float16, device="cuda")
+    y = b2a.attn_block_fwd(torch.from_numpy(x).cuda(), torch.from_numpy(w_qkv).cuda(),
+                           torch.from_numpy(w_o).cuda(), H, d, qkv_ws=qkv_ws, attn_ws=attn_ws, scale=scale,
+                           qknorm=(torch.from_numpy(g_q).cuda(), torch.from_numpy(g_k).cuda(), eps))
+    b2a.check_status()
+    check(qkv_ws.cpu().numpy(), rqkv, "qknorm block qkv")
+    check(attn_ws.cpu().numpy(), ra, "qknorm block attention")
+    check(y.cpu().numpy(), ry, "qknorm block output")
