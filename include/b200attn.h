@@ -323,6 +323,22 @@ B2A_API uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P);
  */
 B2A_API int b2a_check_status(void* stream);
 
+/*
+ * b2a_selftest_wait_timeout -- exercise the failure path without a fault.
+ *
+ * Launches one small kernel on `stream` whose bounded wait (the same code
+ * every kernel here uses for its mbarrier waits) waits on a barrier that
+ * nothing arrives on.  After limit_ms (1..2000) the wait gives up and sets
+ * the device status word, as a lost arrival would; the next
+ * b2a_check_status() returns B2A_ERR_TIMEOUT and clears it.  Until then,
+ * kernels launched afterwards give up at their first wait that does not
+ * complete at once.  result: device int[2], set to {1, 1} when the expired
+ * wait reported failure and a completed wait (checked alongside) reported
+ * success.  The pages have no counterpart; this is for testing callers'
+ * error handling.
+ */
+B2A_API int b2a_selftest_wait_timeout(int limit_ms, int* result, void* stream);
+
 /* Static text for a b2a_status value. */
 B2A_API const char* b2a_status_string(int status);
 

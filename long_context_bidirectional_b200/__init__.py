@@ -26,7 +26,7 @@ __all__ = [
     "attn_merge", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
     "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PAIR",
     "qkv_proj", "qkv_proj_qknorm", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
-    "host_workspace_bytes", "check_status",
+    "host_workspace_bytes", "check_status", "selftest_wait_timeout",
     "chunk_bounds", "library_path",
 ]
 
@@ -57,6 +57,7 @@ _SIGS = {
     "attn_fwd_host": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _i, _vp, ctypes.c_uint64, _vp]),
     "attn_fwd_host_workspace_bytes": (ctypes.c_uint64, [_i, _i, _i, _i]),
     "b2a_check_status": (_i, [_vp]),
+    "b2a_selftest_wait_timeout": (_i, [_i, _vp, _vp]),
     "b2a_status_string": (ctypes.c_char_p, [_i]),
     "b2a_last_cuda_error": (_i, []),
     "b2a_version": (_i, []),
@@ -469,3 +470,14 @@ def attn_fwd_host(q, k, v, out, lse, workspace, P: int = 1, scale=None, stream=N
 def check_status(stream=None) -> None:
     """Synchronise and raise if any kernel reported a device-side timeout."""
     _call("b2a_check_status", _stream(stream))
+
+
+def selftest_wait_timeout(limit_ms: int = 50, stream=None):
+    """Run the failure-path self test; returns the device ``result`` tensor.
+
+    Afterwards :func:`check_status` raises once with B2A_ERR_TIMEOUT (and
+    clears the status).  See ``b2a_selftest_wait_timeout`` in the C header.
+    """
+    result = torch.zeros(2, dtype=torch.int32, device="cuda")
+    _call("b2a_selftest_wait_timeout", int(limit_ms), result.data_ptr(), _stream(stream))
+    return result

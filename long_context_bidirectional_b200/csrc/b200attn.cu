@@ -74,6 +74,34 @@ int current_device(const DeviceInfo** info) {
   return B2A_OK;
 }
 
+// Failure-path self test: thread 0 waits, through the kernels' own bounded
+// wait, on an mbarrier that nothing arrives on; after ``limit_ns`` the wait
+// gives up and sets the status word, exactly as a lost arrival would in an
+// attention or GEMM kernel.  Thread 1 checks a wait that does complete.
+// result[0] = 1 if the first wait reported failure, result[1] = 1 if the
+// second reported success.
+__global__ void selftest_wait_kernel(unsigned int* status, uint64_t limit_ns, int* result) {
+  __shared__ uint64_t bars[2];
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    b2a::mbar_init(b2a::smem_u32(&bars[0]), 1);
+    b2a::mbar_init(b2a::smem_u32(&bars[1]), 1);
+    abort_flag = 0;
+    b2a::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 1) {
+    b2a::mbar_arrive(b2a::smem_u32(&bars[1]));
+    result[1] = b2a::mbar_wait(b2a::smem_u32(&bars[1]), 0, &abort_flag, status) ? 1 : 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool got = b2a::mbar_try_wait(b2a::smem_u32(&bars[0]), 0) ||
+                     b2a::mbar_wait_slow(b2a::smem_u32(&bars[0]), 0, &abort_flag, status, limit_ns);
+    result[0] = got ? 0 : 1;
+  }
+}
+
 // ------------------------------------------------------------ TMA maps ----
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -604,6 +632,17 @@ int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   if (lse && (e = cudaMemcpyAsync(lse, dlse, lbytes, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
     return cuda_fail(e);
   return B2A_OK;
+}
+
+int b2a_selftest_wait_timeout(int limit_ms, int* result, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000 || !result) return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  int st = current_device(&di);
+  if (st != B2A_OK) return st;
+  selftest_wait_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(
+      di->status, static_cast<uint64_t>(limit_ms) * 1000000ull, result);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? B2A_OK : cuda_fail(e);
 }
 
 int b2a_check_status(void* stream) {

@@ -83,7 +83,7 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Slow path of mbar_wait: sleep in try_wait, give up after kWaitLimitNs, on
 // this CTA's abort flag, or when another CTA has set the status word.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                            unsigned int* status) {
+                                            unsigned int* status, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     // sleeps until the phase completes or ~0.1 ms pass
@@ -95,7 +95,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
       *abort_flag = 1;
       return false;
     }
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(status, kDevErrTimeout);
       return false;
