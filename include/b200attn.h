@@ -299,9 +299,17 @@ B2A_API int attn_block_fwd_static(const uint16_t* x, const uint16_t* w_qkv, cons
  * workspace, runs attn_fwd (P == 1) or P attn_fwd_partial calls plus
  * attn_merge (P > 1, the one-device emulation of ring attention), and copies
  * out (host fp16 [S, H, d]) and lse (host fp32 [H, S], may be NULL) back.
- * All copies are cudaMemcpyAsync on `stream`; the call returns after
- * enqueueing, so the host buffers must stay valid until the stream is
- * synchronised.  With page-locked host buffers the copies are asynchronous.
+ * The copies run on two copy streams the library creates on first use per
+ * device (one per direction) so that they overlap the kernels: with P = 1
+ * and S >= 4096 the query rows go in 4 blocks (block b's copy-in, attention
+ * and copy-out overlap the others; K and V are copied first), with P > 1
+ * each key chunk's copy overlaps the previous chunk's partial.  Events order
+ * every step after the work already on `stream` and make `stream` wait for
+ * the last copy-out, so to the caller the call behaves as if enqueued on
+ * `stream`.  The call returns after enqueueing: host buffers must stay valid
+ * until the stream is synchronised.  Page-locked host buffers are needed for
+ * the copies to be asynchronous.  Calls from several host threads on one
+ * device are serialised while they enqueue.
  *
  * workspace        device memory of at least attn_fwd_host_workspace_bytes(S,H,d,P)
  *                  bytes, 256-byte aligned.

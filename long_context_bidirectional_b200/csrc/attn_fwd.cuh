@@ -44,6 +44,7 @@ struct AttnParams {
   int Sq;             // query rows
   int Skv;            // key/value rows
   int H;              // heads
+  int lse_ld;         // row stride of lse / lse_part ([H, lse_ld]); Sq unless a row block
   float scale_log2;   // scale * log2(e)
   uint16_t* out;      // monolithic: fp16 [Sq, ld_o], head h at column h*D;
                       // accumulate: fp16 [Sq, H, D] (ld_o = H*D) or null
@@ -173,7 +174,7 @@ constexpr float kLog2eF = 1.4426950408889634f;
 template <int MODE>
 __device__ __forceinline__ float accum_lse2(const AttnParams& p, int row, int head) {
   if constexpr (MODE == kModeAccum) {
-    if (row < p.Sq) return p.lse_part[static_cast<size_t>(head) * p.Sq + row] * kLog2eF;
+    if (row < p.Sq) return p.lse_part[static_cast<size_t>(head) * p.lse_ld + row] * kLog2eF;
   }
   return -INFINITY;
 }
@@ -250,7 +251,7 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row, int 
     }
   }
   if (live && write_lse) {
-    const size_t li = static_cast<size_t>(head) * p.Sq + row;
+    const size_t li = static_cast<size_t>(head) * p.lse_ld + row;
     if constexpr (MODE == kModeFwd) {
       if (p.lse) p.lse[li] = lse2 * kLn2;
     } else {

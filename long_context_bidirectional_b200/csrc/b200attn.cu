@@ -190,6 +190,7 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   prm.Sq = Sq;
   prm.Skv = Skv;
   prm.H = H;
+  if (prm.lse_ld == 0) prm.lse_ld = Sq;
   prm.scale_log2 = scale * kLog2e;
   auto kern = b2a::attn_fwd_kernel<D, MODE, B2A_ATTN_EMU>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -230,6 +231,7 @@ int launch_attn_pair(const void* q, const void* k, const void* v, int Sq, int Sk
   prm.Sq = Sq;
   prm.Skv = Skv;
   prm.H = H;
+  if (prm.lse_ld == 0) prm.lse_ld = Sq;
   prm.scale_log2 = scale * kLog2e;
   auto kern = b2a::attn_pair_kernel<MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -252,7 +254,7 @@ int launch_any(const void* q, const void* k, const void* v, int Sq, int Skv, int
 
 int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
                   int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_k, int ld_v, int ld_o,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, int lse_ld = 0) {
   if (Skv < 1) return B2A_ERR_INVALID_ARG;
   int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_k, ld_v);
   if (st != B2A_OK) return st;
@@ -264,6 +266,7 @@ int attn_fwd_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   prm.out = out;
   prm.ld_o = ld_o;
   prm.lse = lse;
+  prm.lse_ld = lse_ld;
   prm.status = di->status;
   return launch_any<b2a::kModeFwd>(q, k, v, Sq, Skv, H, d, ld_q, ld_k, ld_v, scale, prm, stream);
 }
@@ -460,6 +463,37 @@ bool host_ws_layout(int S, int H, int d, int P, HostWs* w) {
   return true;
 }
 
+// Copy streams and events of attn_fwd_host, created on first use per device
+// (not memory allocations: two streams and a ring of events).
+struct HostPipe {
+  static constexpr int kEvents = 16;
+  std::mutex mu;  // the event ring is shared: one host caller at a time
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t ev[kEvents] = {};
+  bool ready = false;
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_init_mu;
+constexpr int kHostRowBlock = 1024;  // P = 1 splits the query rows in 4 blocks from 4*1024 rows up
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return B2A_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_pipe_init_mu);
+  HostPipe& hp = g_pipe[dev];
+  if (!hp.ready) {
+    if ((e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking)) != cudaSuccess) return cuda_fail(e);
+    for (int i = 0; i < HostPipe::kEvents; ++i)
+      if ((e = cudaEventCreateWithFlags(&hp.ev[i], cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+    hp.ready = true;
+  }
+  *out = &hp;
+  return B2A_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -596,6 +630,9 @@ int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   const DeviceInfo* di = nullptr;
   int st = current_device(&di);
   if (st != B2A_OK) return st;
+  HostPipe* hp = nullptr;
+  if ((st = host_pipe(&hp)) != B2A_OK) return st;
+  std::lock_guard<std::mutex> lk(hp->mu);
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint16_t* dq = reinterpret_cast<uint16_t*>(ws + w.q);
@@ -603,34 +640,79 @@ int attn_fwd_host(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint1
   uint16_t* dv = reinterpret_cast<uint16_t*>(ws + w.v);
   uint16_t* dout = reinterpret_cast<uint16_t*>(ws + w.out);
   float* dlse = reinterpret_cast<float*>(ws + w.lse);
-  const size_t nbytes = static_cast<size_t>(S) * H * d * 2;
-  const size_t lbytes = static_cast<size_t>(S) * H * 4;
-  cudaError_t e;
-  if ((e = cudaMemcpyAsync(dq, q, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
-  if ((e = cudaMemcpyAsync(dk, k, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
-  if ((e = cudaMemcpyAsync(dv, v, nbytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess) return cuda_fail(e);
   const int ld = H * d;
+  const size_t row16 = static_cast<size_t>(ld) * 2;  // bytes of one fp16 row
+  cudaError_t e;
+  int ev = 0;
+  // signal ``from`` -> ``to`` through the next event of the ring: every wait
+  // is enqueued before that event is recorded again, so reuse is safe
+  auto handoff = [&](cudaStream_t from, cudaStream_t to) -> cudaError_t {
+    cudaEvent_t x = hp->ev[ev++ % HostPipe::kEvents];
+    cudaError_t r = cudaEventRecord(x, from);
+    return r == cudaSuccess ? cudaStreamWaitEvent(to, x, 0) : r;
+  };
+  // Copies run on the library's own two copy streams (one per direction) so
+  // that they overlap the kernels on ``stream``; events keep every step in
+  // order with the caller's earlier and later work on ``stream``.
+  if ((e = handoff(stream, hp->h2d)) != cudaSuccess) return cuda_fail(e);
+  if ((e = handoff(stream, hp->d2h)) != cudaSuccess) return cuda_fail(e);
   if (P == 1) {
-    st = attn_fwd_impl(dq, dk, dv, dout, dlse, S, S, H, d, scale, ld, ld, ld, ld, stream);
+    // K and V first (every query row needs all of them), then query rows in
+    // blocks: block b's copy-in, attention and copy-out overlap the others.
+    if ((e = cudaMemcpyAsync(dk, k, S * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(dv, v, S * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess) return cuda_fail(e);
+    const int nb = S >= 4 * kHostRowBlock ? 4 : 1;
+    for (int b = 0; b < nb; ++b) {
+      const int r0 = static_cast<int>(static_cast<long long>(b) * S / nb);
+      const int r1 = static_cast<int>(static_cast<long long>(b + 1) * S / nb);
+      const size_t off = static_cast<size_t>(r0) * ld;
+      if ((e = cudaMemcpyAsync(dq + off, q + off, (r1 - r0) * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess)
+        return cuda_fail(e);
+      if ((e = handoff(hp->h2d, stream)) != cudaSuccess) return cuda_fail(e);
+      st = attn_fwd_impl(dq + off, dk, dv, dout + off, dlse + r0, r1 - r0, S, H, d, scale, ld, ld, ld, ld, stream, S);
+      if (st != B2A_OK) return st;
+      if ((e = handoff(stream, hp->d2h)) != cudaSuccess) return cuda_fail(e);
+      if ((e = cudaMemcpyAsync(out + off, dout + off, (r1 - r0) * row16, cudaMemcpyDeviceToHost, hp->d2h)) !=
+          cudaSuccess)
+        return cuda_fail(e);
+      if (lse && (e = cudaMemcpy2DAsync(lse + r0, static_cast<size_t>(S) * 4, dlse + r0, static_cast<size_t>(S) * 4,
+                                        static_cast<size_t>(r1 - r0) * 4, H, cudaMemcpyDeviceToHost, hp->d2h)) !=
+                     cudaSuccess)
+        return cuda_fail(e);
+    }
   } else {
+    // Ring-attention emulation: Q first, then each key chunk's K/V copy
+    // overlaps the previous chunk's partial.
     float* op = reinterpret_cast<float*>(ws + w.o_parts);
     float* lp = reinterpret_cast<float*>(ws + w.lse_parts);
     const size_t n = static_cast<size_t>(S) * H * d;
     const size_t nl = static_cast<size_t>(S) * H;
-    st = B2A_OK;
-    for (int c = 0; c < P && st == B2A_OK; ++c) {
+    if ((e = cudaMemcpyAsync(dq, q, S * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess) return cuda_fail(e);
+    for (int c = 0; c < P; ++c) {
       const long long lo = static_cast<long long>(c) * S / P;
       const long long hi = static_cast<long long>(c + 1) * S / P;
-      st = attn_partial_impl(dq, dk + lo * ld, dv + lo * ld, op + c * n, lp + c * nl, S,
-                             static_cast<int>(hi - lo), H, d, scale, ld, ld, stream);
+      const size_t off = static_cast<size_t>(lo) * ld;
+      if (hi > lo) {
+        if ((e = cudaMemcpyAsync(dk + off, k + off, (hi - lo) * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess)
+          return cuda_fail(e);
+        if ((e = cudaMemcpyAsync(dv + off, v + off, (hi - lo) * row16, cudaMemcpyHostToDevice, hp->h2d)) != cudaSuccess)
+          return cuda_fail(e);
+      }
+      if ((e = handoff(hp->h2d, stream)) != cudaSuccess) return cuda_fail(e);
+      st = attn_partial_impl(dq, dk + off, dv + off, op + c * n, lp + c * nl, S, static_cast<int>(hi - lo), H, d,
+                             scale, ld, ld, stream);
+      if (st != B2A_OK) return st;
     }
-    if (st == B2A_OK) st = attn_merge_impl(op, lp, P, dout, dlse, S, H, d, stream);
+    if ((st = attn_merge_impl(op, lp, P, dout, dlse, S, H, d, stream)) != B2A_OK) return st;
+    if ((e = handoff(stream, hp->d2h)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaMemcpyAsync(out, dout, S * row16, cudaMemcpyDeviceToHost, hp->d2h)) != cudaSuccess)
+      return cuda_fail(e);
+    if (lse && (e = cudaMemcpyAsync(lse, dlse, static_cast<size_t>(S) * H * 4, cudaMemcpyDeviceToHost, hp->d2h)) !=
+                   cudaSuccess)
+      return cuda_fail(e);
   }
-  if (st != B2A_OK) return st;
-  if ((e = cudaMemcpyAsync(out, dout, nbytes, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
-    return cuda_fail(e);
-  if (lse && (e = cudaMemcpyAsync(lse, dlse, lbytes, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
-    return cuda_fail(e);
+  // the caller's stream resumes after the last copy-out
+  if ((e = handoff(hp->d2h, stream)) != cudaSuccess) return cuda_fail(e);
   return B2A_OK;
 }
 

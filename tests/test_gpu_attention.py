@@ -221,17 +221,37 @@ def test_seq8k_h64_workload_sampled(b2a):
     _sampled_check(b2a, W.SEQ8K_H64, 1)
 
 
-def test_host_entry_point_end_to_end(b2a):
-    S, H, d = 1000, 2, 128
+@pytest.mark.parametrize("S", [1000, 4500])
+def test_host_entry_point_end_to_end(b2a, S):
+    # S = 4500: the P = 1 path copies and computes the query rows in 4 blocks
+    # (row-strided LSE copies), the chunked path copies each key chunk
+    # while the previous chunk's partial runs
+    H, d = 2, 128
     q, k, v = W.qkv(S, H, d, seed=14)
     scale = 1 / math.sqrt(d)
     ref, ref_lse = OA.attention(q, k, v, scale)
-    for P in (1, 3):
+    for P in (1, 3, 8):
         ws = torch.empty(b2a.host_workspace_bytes(S, H, d, P), dtype=torch.uint8, device="cuda")
         qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
         out = torch.empty((S, H, d), dtype=torch.float16).pin_memory()
         lse = torch.empty((H, S), dtype=torch.float32).pin_memory()
         b2a.attn_fwd_host(qh, kh, vh, out, lse, ws, P=P, scale=scale)
         b2a.check_status()
-        assert_out_close(out.numpy().astype(np.float64), ref, f"host P={P}")
+        assert_out_close(out.numpy().astype(np.float64), ref, f"host S={S} P={P}")
         assert_lse_close(lse.numpy(), ref_lse)
+    # two calls back to back on one stream, no sync between: the second's
+    # copies must wait for the first's use of the shared workspace
+    ws = torch.empty(b2a.host_workspace_bytes(S, H, d, 4), dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((S, H, d), dtype=torch.float16).pin_memory() for _ in range(2)]
+    lses = [torch.empty((H, S), dtype=torch.float32).pin_memory() for _ in range(2)]
+    q2 = q.copy()
+    q2[:, 0] = q[:, 1]  # a different second call
+    ref2, ref2_lse = OA.attention(q2, k, v, scale)
+    kh, vh = torch.from_numpy(k).pin_memory(), torch.from_numpy(v).pin_memory()
+    qhs = [torch.from_numpy(qq).pin_memory() for qq in (q, q2)]   # alive until the sync below
+    for i, P in enumerate((1, 4)):
+        b2a.attn_fwd_host(qhs[i], kh, vh, outs[i], lses[i], ws, P=P, scale=scale)
+    b2a.check_status()
+    assert_out_close(outs[0].numpy().astype(np.float64), ref, "host back-to-back 1")
+    assert_out_close(outs[1].numpy().astype(np.float64), ref2, "host back-to-back 2")
+    assert_lse_close(lses[1].numpy(), ref2_lse)
