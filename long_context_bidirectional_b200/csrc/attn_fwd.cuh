@@ -8,7 +8,11 @@
 // 128-wide tiles with an online (running-max) softmax, the form ring
 // attention relies on (TensorRT 11.0 multi-device article, Ring Attention).
 //
-// Used for head dim 64 (head dim 128 runs on CTA pairs, attn_pair.cuh).
+// Used for head dim 64, and for head dim 128 when a call has fewer than 96
+// key tiles (longer key ranges run on CTA pairs, attn_pair.cuh: this kernel's
+// pipeline fills and drains in fewer SM-cycles per row).  Both write their
+// results through attn_epilogue below, in the monolithic, partial or
+// accumulate (ring step) form.
 // One CTA owns two 128-row query tiles of one head.  Warp roles (18 warps):
 //   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1.  Each
 //               row is shared by two threads (warps w and w+4 of a group, the

@@ -1,6 +1,7 @@
-// Non-causal attention forward on CTA pairs (sm_100a, head dim 128).
+// Non-causal attention forward on CTA pairs (sm_100a, head dim 128, calls
+// with at least 96 key tiles unless chosen explicitly).
 //
-// Same result as attn_fwd_kernel (per head and query row: the softmax of the
+// Same result as attn_fwd_kernel, bit for bit (per head and query row: the softmax of the
 // scaled logits against every key, times V, and the natural-log LSE: "Multi-
 // Device Attention Inference with TensorRT", Introduction; "Tensor
 // Parallelism: Sharding Weights for Parallel Layer Execution", section 3),
@@ -20,15 +21,17 @@
 // | O (4 x 128 columns).  The softmax writes P(j) (fp16) over S[j%3] and PV(j)
 // reads it there; in-order tcgen05 execution keeps P(j) alive until PV(j)
 // has read it, so the leader issues S(j+3) = Q K(j+3)^T into the same buffer
-// right behind PV(j):
-//   QK(0) QK(1) QK(2) | PV(0) QK(3) | PV(1) QK(4) | ...
+// once PV(j) has completed:
+//   QK(0) QK(1) QK(2) | PV(0) -> QK(3) | PV(1) -> QK(4) | ...
+// (PVs and QKs come from two issuing threads; see the PV issuer below).
 // Each CTA's softmax therefore finds the scores of its next two tiles
 // already computed and runs tile after tile; the P-ready -> PV -> QK -> S
 // chain has two softmax periods to complete instead of one.
-// Warp roles per CTA (11 warps): warps 0-7 softmax (each row shared by two
+// Warp roles per CTA (12 warps): warps 0-7 softmax (each row shared by two
 // threads, 64 score columns each, row max exchanged through shared memory),
-// warp 8 TMA producer, warp 9 TMEM allocator and (leader only) MMA issuer,
-// warp 10 (leader only) waits on the MMAs' input barriers for the issuer.
+// warp 8 TMA producer, warp 9 TMEM allocator and (leader only) PV issuer,
+// warp 10 (leader only) waits for P on the PV issuer's behalf, warp 11
+// (leader only) QK issuer.
 // Barriers the MMAs depend on (Q and K/V arrival, P ready) live in the
 // leader; barriers the MMAs signal (score ready, slot free = PV done) are
 // signalled in both CTAs by multicast commits.  The P-ready arrivals that
@@ -67,16 +70,17 @@ struct AttnPairShape {
   static constexpr int B_S = 1 + 2 * STAGES;
   static constexpr int B_P = B_S + NSB;
   static constexpr int B_OF = B_P + NSB;
-  static constexpr int B_DRAIN = B_OF + 1;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_OF + 1;    // the PV issuer's last commit
+  static constexpr int B_DRAIN2 = B_DRAIN + 1;  // the QK issuer's last commit
+  static constexpr int NBAR = B_DRAIN2 + 1;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;           // [parity][half][row] floats
   static constexpr int OFF_LSUM = OFF_RED + 2 * 2 * BM * 4;    // [row] floats
   static constexpr int OFF_MISC = OFF_LSUM + BM * 4;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr int TM_O = NSB * 128;
   static constexpr int TM_COLS = 512;
-  static constexpr int THREADS = 352;
-  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SYNC = 10;
+  static constexpr int THREADS = 384;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SYNC = 10, WARP_QK = 11;
   static constexpr int BAR_HANDOFF = 5;    // named barrier: MMA warp + helper warp
   static constexpr int P_ARRIVALS = 16;                        // 8 softmax warps x 2 CTAs
   static constexpr int ROWS_PER_PAIR = 2 * BM;
@@ -86,7 +90,7 @@ struct AttnPairShape {
 };
 
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -130,6 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     }
     mbar_init(bar(C::B_OF), 1);
     mbar_init(bar(C::B_DRAIN), 1);
+    mbar_init(bar(C::B_DRAIN2), 1);
     // A CTA launched after an earlier one timed out gives up at its first
     // wait that does not complete at once.
     *abort_flag = (*reinterpret_cast<volatile unsigned int*>(p.status) != 0u) ? 1 : 0;
@@ -183,21 +188,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
     }
     __syncwarp();
   } else if (warp == C::WARP_MMA) {
-    // ------------------------------------------------------- MMA issuer --
-    // The issuing thread polls no mbarrier itself: a synchronising
-    // instruction it executes (a barrier poll, even a shared-memory read)
-    // waits behind the MMAs it has queued while the tensor core drains.  The
-    // helper warp waits for P(j) and K/V(j+NSB) instead, and the two warps
-    // meet at a named barrier per tile (which also carries whether to go on;
-    // measured at ~300 issue cycles, against ~600 for the issuer's own
-    // polls).  Handing over two tiles per meeting was measured too: it
-    // starves the softmax, which then waits for S(j+3) behind P(j+1).
+    // --------------------------------------------------- PV issuer (leader) --
+    // The MMAs come from two threads (tcgen05.mma from several threads is
+    // unordered between them, ordered within each).  This one issues PV(j)
+    // into O; warp WARP_QK issues QK(j+3) into S[j%3] once PV(j) has read
+    // P(j) from there (its kv_empty commit).  A synchronising instruction of
+    // an issuing thread (a barrier poll, a named barrier) waits behind the
+    // MMAs it has queued while the tensor core drains, so with one issuer
+    // every poll left a gap; with two, each fills the other's gaps (probe:
+    // 1438 -> 1172 cycles per tile with no softmax work).  The helper warp
+    // waits for P(j) for this thread, and the two meet at a named barrier
+    // per tile (which also carries whether to go on).
     if (leader) {
-      constexpr uint32_t idesc_qk = idesc_f16_f32(256, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_f16_f32(256, D, false, true);
-      const uint64_t dq = sw128_desc(sQ, 16, 1024);                      // Q, K-major
-      const uint64_t dk = sw128_desc(sKV, 16, 1024);                     // K half, K-major
       const uint64_t dv = sw128_desc(sKV + C::KH_BYTES, C::KSUB, 1024);  // V half, MN-major
+      auto issue_pv = [&](int buf, int st, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_ts_pair(tmem + C::TM_O, tmem + C::tm_s(buf) + kk * 8,
+                      dv + ((st * C::STAGE_BYTES + kk * 2048) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
+      };
+      // score buffer and K/V stage of tile j
+      int buf = 0, st = 0;
+      for (int j = 0; j < nkv; ++j) {
+        if (!pair_barrier_and(C::BAR_HANDOFF, true)) break;
+        if (lane == 0) {
+          tc_fence_after();
+          B2A_TR(kTrPv0Issue, j);
+          issue_pv(buf, st, j > 0);
+          // PV(j) done: K(j)/V(j) consumed, P(j)'s buffer free for QK(j+3),
+          // and O holds PV(0..j) for the softmax's rescale
+          tc_commit_pair(bar(C::B_KVE + st));
+          if (j + 1 == nkv) tc_commit_pair(bar(C::B_OF));
+          B2A_TR(kTrPv0Done, j);
+        }
+        __syncwarp();
+        if (++buf == C::NSB) buf = 0;
+        if (++st == C::STAGES) st = 0;
+      }
+      if (lane == 0) {
+        // Every MMA this thread issued must finish before TMEM is released.
+        tc_commit_pair(bar(C::B_DRAIN));
+        mbar_drain(bar(C::B_DRAIN), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == C::WARP_QK) {
+    // --------------------------------------------------- QK issuer (leader) --
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_f16_f32(256, 128, false, false);
+      const uint64_t dq = sw128_desc(sQ, 16, 1024);   // Q, K-major
+      const uint64_t dk = sw128_desc(sKV, 16, 1024);  // K half, K-major
       auto issue_qk = [&](int buf, int st) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -206,72 +247,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
           mma_ss_pair(tmem + C::tm_s(buf), dq + (qoff >> 4), dk + (koff >> 4), idesc_qk, kk > 0);
         }
       };
-      auto issue_pv = [&](int buf, int st, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_ts_pair(tmem + C::TM_O, tmem + C::tm_s(buf) + kk * 8,
-                      dv + ((st * C::STAGE_BYTES + kk * 2048) >> 4), idesc_pv, (acc || kk > 0) ? 1u : 0u);
-      };
-      int ok = 1;
-      if (lane == 0) {
-        ok = mbar_wait(bar(C::B_Q), 0, abort_flag, p.status);
-        for (int j = 0; j < C::NSB && j < nkv && ok; ++j) {
-          if (!(ok = mbar_wait(bar(C::B_KVF + j % C::STAGES), (j / C::STAGES) & 1, abort_flag, p.status))) break;
-          tc_fence_after();
-          issue_qk(j, j % C::STAGES);
-          tc_commit_pair(bar(C::B_S + j));
-        }
+      bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, p.status);
+      for (int j = 0; j < C::NSB && j < nkv && ok; ++j) {
+        if (!(ok = mbar_wait(bar(C::B_KVF + j % C::STAGES), (j / C::STAGES) & 1, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_qk(j, j % C::STAGES);
+        tc_commit_pair(bar(C::B_S + j));
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      // score buffer and K/V stage of tile j; the stage of tile j + NSB
-      int buf = 0, st = 0, st3 = C::NSB % C::STAGES;
-      for (int j = 0; j < nkv; ++j) {
-        if (!pair_barrier_and(C::BAR_HANDOFF, ok != 0)) break;
-        if (lane == 0) {
-          tc_fence_after();
-          B2A_TR(kTrPv0Issue, j);
-          issue_pv(buf, st, j > 0);
-          // K(j) and V(j) consumed; also tells the softmax that O holds PV(j)
-          tc_commit_pair(bar(C::B_KVE + st));
-          if (j + 1 == nkv) tc_commit_pair(bar(C::B_OF));
-          B2A_TR(kTrPv0Done, j);
-          if (j + C::NSB < nkv) {
-            issue_qk(buf, st3);
-            tc_commit_pair(bar(C::B_S + buf));
-          }
-          B2A_TR(kTrQk0Issue, j);
-        }
-        __syncwarp();
+      // QK(j+3) into S[j%3] after PV(j) (kv_empty of tile j's stage: it
+      // cannot be a phase ahead, PV(j+STAGES) needs QK(j+STAGES) from this
+      // thread) and K(j+3)'s arrival
+      int buf = 0, st = 0, sph = 0, st3 = C::NSB % C::STAGES, sph3 = (C::NSB / C::STAGES) & 1;
+      for (int j = 0; j + C::NSB < nkv && ok; ++j) {
+        if (!(ok = mbar_wait(bar(C::B_KVE + st), sph, abort_flag, p.status))) break;
+        if (!(ok = mbar_wait(bar(C::B_KVF + st3), sph3, abort_flag, p.status))) break;
+        tc_fence_after();
+        issue_qk(buf, st3);
+        tc_commit_pair(bar(C::B_S + buf));
+        B2A_TR(kTrQk0Issue, j);
         if (++buf == C::NSB) buf = 0;
-        if (++st == C::STAGES) st = 0;
-        if (++st3 == C::STAGES) st3 = 0;
+        if (++st == C::STAGES) { st = 0; sph ^= 1; }
+        if (++st3 == C::STAGES) { st3 = 0; sph3 ^= 1; }
       }
-      if (lane == 0) {
-        // Every MMA issued above must finish before TMEM is released.
-        tc_commit_pair(bar(C::B_DRAIN));
-        mbar_drain(bar(C::B_DRAIN), 0);
-      }
+      // every QK this thread issued must finish before TMEM is released
+      tc_commit_pair(bar(C::B_DRAIN2));
+      mbar_drain(bar(C::B_DRAIN2), 0);
     }
     __syncwarp();
   } else if (warp == C::WARP_SYNC) {
     // ---------------------------------------------- helper (leader only) --
     if (leader) {
       int bph = 0, buf = 0;
-      int st3 = C::NSB % C::STAGES, sph3 = (C::NSB / C::STAGES) & 1;
       for (int j = 0; j < nkv; ++j) {
         int ok = 1;
         if (lane == 0) {
           B2A_TR(kTrSlotWait, j);
-          if (j + C::NSB < nkv) ok = mbar_wait(bar(C::B_KVF + st3), sph3, abort_flag, p.status);
           // arrivals from the other CTA do not wake a suspended try_wait
           // promptly: poll without suspending
-          if (ok) ok = mbar_spin(bar(C::B_P + buf), bph, abort_flag, p.status);
+          ok = mbar_spin(bar(C::B_P + buf), bph, abort_flag, p.status);
           B2A_TR(kTrSlotReady, j);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!pair_barrier_and(C::BAR_HANDOFF, ok != 0)) break;
         if (++buf == C::NSB) { buf = 0; bph ^= 1; }
-        if (++st3 == C::STAGES) { st3 = 0; sph3 ^= 1; }
       }
     }
     __syncwarp();
@@ -436,7 +454,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(352, 1)
   // The drain commit also lands in the peer: wait for it there before the
   // CTA can exit.  (Not earlier: a thread polling a barrier for the whole
   // kernel slows the pair's tensor-core work on that SM.)
-  if (!leader && warp == C::WARP_MMA && lane == 0) mbar_drain(bar(C::B_DRAIN), 0);
+  if (!leader && warp == C::WARP_MMA && lane == 0) {
+    mbar_drain(bar(C::B_DRAIN), 0);
+    mbar_drain(bar(C::B_DRAIN2), 0);
+  }
   // neither CTA releases TMEM or exits while the pair's MMAs or loads may
   // still touch its TMEM, shared memory or barriers
   cluster_sync();
