@@ -370,6 +370,22 @@ def run_ours(args, rank, world, local):
                                              scale=w.scale, stream=stream))
     del cp_out
 
+    # The FP16 split-reduction: the same P partials stored in fp16, and the
+    # merge reading them (half the partial bytes).  Not part of ``value``.
+    o16_parts = torch.empty((P, S, H, d), dtype=torch.float16, device=dev)
+
+    def part16_pass():
+        for c, (c_lo, c_hi) in enumerate(bounds):
+            b2a.attn_fwd_partial_f16(qd, kd[c_lo:c_hi], vd[c_lo:c_hi], o16_parts[c], lse_parts[c],
+                                     scale=w.scale, stream=stream)
+
+    p16_ms = time_calls(part16_pass, n=3)
+    m16_ms = time_calls(lambda: b2a.attn_merge_f16(o16_parts, lse_parts, out=out_c, lse_out=lse_c,
+                                                   stream=stream))
+    del o16_parts
+    merge16_bytes = P * S * H * d * 2 + P * H * S * 4 + S * H * d * 2 + H * S * 4
+    merge16_gbs = merge16_bytes / (m16_ms * 1e-3) / 1e9
+
     # end to end from pinned host memory through the C-ABI host entry point
     e2e = None
     if not args.no_e2e:
@@ -443,7 +459,12 @@ def run_ours(args, rank, world, local):
                     "cp_ulysses_rank_tflops": 4.0 * S * S * d * nh / (uly_ms * 1e-3) / 1e12,
                     "cp_ranks": f"8-way: AllGather-KV rank 3 ({hi - lo} rows x {S} keys), Ulysses rank 3 "
                                 f"({nh} of {H} heads); not in value",
-                    "merge_hbm_frac": merge_gbs / pk["hbm_gbs"], "merge_bytes": merge_bytes},
+                    "merge_hbm_frac": merge_gbs / pk["hbm_gbs"], "merge_bytes": merge_bytes,
+                    "fp16_partial_pass_ms": p16_ms,
+                    "fp16_partial_pass_tflops": w.flops / (p16_ms * 1e-3) / 1e12,
+                    "merge_f16_ms": m16_ms, "merge_f16_gbs": merge16_gbs,
+                    "merge_f16_hbm_frac": merge16_gbs / pk["hbm_gbs"], "merge_f16_bytes": merge16_bytes,
+                    "fp16_split_reduction": f"{P} x attn_fwd_partial_f16 + attn_merge_f16 (not in value)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * (P + 2),

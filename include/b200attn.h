@@ -131,6 +131,22 @@ B2A_API int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const u
                      int ld_q, int ld_kv, void* stream);
 
 /*
+ * attn_fwd_partial_f16 -- attn_fwd_partial with the partial output stored in
+ * fp16: the "FP16 split-reduction" that the accuracy table of "TensorRT
+ * Multi-Device (multi-GPU) support" (Validation) names as the source of its
+ * multi-device error.  o_part = round_fp16(o_c) where o_c is the chunk's
+ * normalised output computed in fp32; lse_part stays fp32.  Half the bytes
+ * of attn_fwd_partial's o_part, which attn_merge_f16 reads back.
+ *
+ * o_part    device fp16 [Sq, H, d], contiguous, 16-byte aligned.
+ * Every other argument, the empty chunk (o_part = 0, lse_part = -inf) and
+ * the error behaviour as attn_fwd_partial.
+ */
+B2A_API int attn_fwd_partial_f16(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
+                                 uint16_t* o_part, float* lse_part, int Sq, int Skv, int H, int d, float scale,
+                                 int ld_q, int ld_kv, void* stream);
+
+/*
  * attn_fwd_accumulate -- one ring-attention step in place: fold the keys of
  * one chunk into a running result, the way each rank of ring attention
  * updates its output as K/V blocks arrive (TensorRT 11.0 multi-device
@@ -174,6 +190,17 @@ B2A_API int attn_fwd_accumulate(const uint16_t* q, const uint16_t* k_chunk, cons
  */
 B2A_API int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
                int S, int H, int d, void* stream);
+
+/*
+ * attn_merge_f16 -- attn_merge over fp16 partials (attn_fwd_partial_f16's
+ * o_part): the same weights and lse in fp32, the partial values widened to
+ * fp32 before the weighted sum, one rounding of the result to fp16.
+ *
+ * o_parts    device fp16 [P, S, H, d] contiguous, 16-byte aligned.
+ * Every other argument and the error behaviour as attn_merge.
+ */
+B2A_API int attn_merge_f16(const uint16_t* o_parts, const float* lse_parts, int P, uint16_t* out,
+                           float* lse_out, int S, int H, int d, void* stream);
 
 /*
  * qkv_proj -- fused Q/K/V projection qkv = x * w_qkv^T ("Tensor Parallelism:

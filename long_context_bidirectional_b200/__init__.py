@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "lib
 
 __all__ = [
     "B2AError", "lib", "attn_fwd", "attn_fwd_batched", "attn_fwd_gathered_kv", "attn_fwd_partial", "attn_fwd_accumulate",
-    "attn_merge", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
+    "attn_fwd_partial_f16", "attn_merge", "attn_merge_f16", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
     "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PAIR",
     "qkv_proj", "qkv_proj_qknorm", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
     "host_workspace_bytes", "check_status", "selftest_wait_timeout",
@@ -48,6 +48,8 @@ _SIGS = {
     "b2a_get_attn_kernel": (_i, []),
     "b2a_attn_kernel_for": (_i, [_i, _i]),
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
+    "attn_fwd_partial_f16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_merge_f16": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "attn_block_fwd_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
@@ -205,6 +207,15 @@ def attn_fwd_gathered_kv(q, k, v, out=None, lse=None, scale=None, return_lse=Tru
 
 def attn_fwd_partial(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None, stream=None):
     """Attention of all queries against one key chunk; returns ``(o_part, lse_part)``."""
+    return _partial("attn_fwd_partial", torch.float32, q, k_chunk, v_chunk, o_part, lse_part, scale, stream)
+
+
+def attn_fwd_partial_f16(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None, stream=None):
+    """``attn_fwd_partial`` with ``o_part`` stored in fp16 (the FP16 split-reduction)."""
+    return _partial("attn_fwd_partial_f16", torch.float16, q, k_chunk, v_chunk, o_part, lse_part, scale, stream)
+
+
+def _partial(fn, odt, q, k_chunk, v_chunk, o_part, lse_part, scale, stream):
     Sq, H, d = q.shape
     ld_q = _check_qkv("q", q)
     Skv = k_chunk.shape[0]
@@ -215,17 +226,17 @@ def attn_fwd_partial(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=None
     if ld_k != ld_v:
         raise ValueError("k_chunk and v_chunk must share a row stride")
     if o_part is None:
-        o_part = torch.empty((Sq, H, d), dtype=torch.float32, device=q.device)
+        o_part = torch.empty((Sq, H, d), dtype=odt, device=q.device)
     if lse_part is None:
         lse_part = torch.empty((H, Sq), dtype=torch.float32, device=q.device)
-    if not (o_part.is_contiguous() and o_part.dtype == torch.float32 and o_part.numel() == Sq * H * d):
-        raise ValueError("o_part must be contiguous float32 [Sq, H, d]")
+    if not (o_part.is_contiguous() and o_part.dtype == odt and o_part.numel() == Sq * H * d):
+        raise ValueError(f"o_part must be contiguous {odt} [Sq, H, d]")
     if not (lse_part.is_contiguous() and lse_part.dtype == torch.float32 and lse_part.numel() == H * Sq):
         raise ValueError("lse_part must be contiguous float32 [H, Sq]")
     # An empty chunk may be a zero-length view; any valid address will do.
     kp = k_chunk.data_ptr() if Skv > 0 else q.data_ptr()
     vp = v_chunk.data_ptr() if Skv > 0 else q.data_ptr()
-    _call("attn_fwd_partial", q.data_ptr(), kp, vp, o_part.data_ptr(), lse_part.data_ptr(),
+    _call(fn, q.data_ptr(), kp, vp, o_part.data_ptr(), lse_part.data_ptr(),
           Sq, Skv, H, d, _default_scale(d, scale), ld_q, ld_k if Skv > 0 else ld_q, _stream(stream))
     return o_part, lse_part
 
@@ -293,9 +304,18 @@ def attn_kernel_for(d: int, Skv: int) -> int:
 
 
 def attn_merge(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stream=None):
-    """Exact merge of partials ``o_parts [P,S,H,d]``, ``lse_parts [P,H,S]``."""
-    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
-        raise TypeError("o_parts and lse_parts must be float32")
+    """Exact merge of partials ``o_parts [P,S,H,d]`` (fp32), ``lse_parts [P,H,S]``."""
+    return _merge("attn_merge", torch.float32, o_parts, lse_parts, out, lse_out, return_lse, stream)
+
+
+def attn_merge_f16(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stream=None):
+    """``attn_merge`` over fp16 partials (``attn_fwd_partial_f16``'s output)."""
+    return _merge("attn_merge_f16", torch.float16, o_parts, lse_parts, out, lse_out, return_lse, stream)
+
+
+def _merge(fn, odt, o_parts, lse_parts, out, lse_out, return_lse, stream):
+    if o_parts.dtype != odt or lse_parts.dtype != torch.float32:
+        raise TypeError(f"o_parts must be {odt} and lse_parts float32")
     if not (o_parts.is_contiguous() and lse_parts.is_contiguous()):
         raise ValueError("o_parts and lse_parts must be contiguous")
     P, S, H, d = o_parts.shape
@@ -307,7 +327,7 @@ def attn_merge(o_parts, lse_parts, out=None, lse_out=None, return_lse=True, stre
         raise ValueError("out must be contiguous float16 [S, H, d]")
     if lse_out is None and return_lse:
         lse_out = torch.empty((H, S), dtype=torch.float32, device=o_parts.device)
-    _call("attn_merge", o_parts.data_ptr(), lse_parts.data_ptr(), P, out.data_ptr(), _ptr(lse_out),
+    _call(fn, o_parts.data_ptr(), lse_parts.data_ptr(), P, out.data_ptr(), _ptr(lse_out),
           S, H, d, _stream(stream))
     return out, lse_out
 
@@ -318,20 +338,26 @@ def chunk_bounds(S: int, P: int):
 
 
 def attn_chunked(q, k, v, P: int, out=None, lse=None, scale=None, o_parts=None, lse_parts=None,
-                 stream=None):
+                 stream=None, partial_dtype=torch.float32):
     """Ring attention emulated on one device: P key-chunk partials, then the merge.
 
-    ``o_parts``/``lse_parts`` are the caller's workspace (allocated here when
-    omitted).  Returns ``(out, lse)``.
+    ``partial_dtype`` float32 (default) or float16 (the FP16 split-reduction:
+    ``attn_fwd_partial_f16`` + ``attn_merge_f16``).  ``o_parts``/``lse_parts``
+    are the caller's workspace (allocated here when omitted).  Returns ``(out, lse)``.
     """
     S, H, d = q.shape
+    if partial_dtype not in (torch.float32, torch.float16):
+        raise ValueError("partial_dtype must be torch.float32 or torch.float16")
+    f16 = partial_dtype == torch.float16
     if o_parts is None:
-        o_parts = torch.empty((P, S, H, d), dtype=torch.float32, device=q.device)
+        o_parts = torch.empty((P, S, H, d), dtype=partial_dtype, device=q.device)
     if lse_parts is None:
         lse_parts = torch.empty((P, H, S), dtype=torch.float32, device=q.device)
+    part = attn_fwd_partial_f16 if f16 else attn_fwd_partial
     for c, (lo, hi) in enumerate(chunk_bounds(k.shape[0], P)):
-        attn_fwd_partial(q, k[lo:hi], v[lo:hi], o_parts[c], lse_parts[c], scale=scale, stream=stream)
-    return attn_merge(o_parts, lse_parts, out=out, lse_out=lse, stream=stream)
+        part(q, k[lo:hi], v[lo:hi], o_parts[c], lse_parts[c], scale=scale, stream=stream)
+    merge = attn_merge_f16 if f16 else attn_merge
+    return merge(o_parts, lse_parts, out=out, lse_out=lse, stream=stream)
 
 
 def _check_mat(name, t, rows=None, cols=None):

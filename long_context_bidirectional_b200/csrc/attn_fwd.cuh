@@ -634,10 +634,11 @@ __global__ void attn_accum_empty_kernel(const float* o_acc, const float* lse_acc
 }
 
 // Fill for an empty key chunk: o = 0, lse = -inf (the empty sum).
-__global__ void attn_empty_partial_kernel(float* o_part, float* lse_part, size_t n_o, size_t n_lse) {
+template <typename T>  // float or uint16_t (fp16 zero is all-zero bits)
+__global__ void attn_empty_partial_kernel(T* o_part, float* lse_part, size_t n_o, size_t n_lse) {
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_o; i += stride)
-    o_part[i] = 0.f;
+    o_part[i] = T(0);
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n_lse; i += stride)
     lse_part[i] = -INFINITY;
 }

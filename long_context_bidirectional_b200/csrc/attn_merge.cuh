@@ -12,22 +12,48 @@
 // One block owns 256 consecutive (s, h) pairs.  Phase 1: thread t computes
 // the P weights of pair t into shared memory and writes lse.  Phase 2: the
 // block streams the pairs' o_p rows, which are contiguous in the
-// [P][S][H][D] layout, as float4 loads (8 chunks in flight per thread),
-// accumulates in fp32 and stores fp16.
+// [P][S][H][D] layout, as 16-byte loads (4 fp32 or 8 fp16 partial values;
+// 8 chunks in flight per thread), accumulates in fp32 and stores fp16.  The
+// fp16 form reads the partials the FP16 split-reduction stores: half the
+// bytes of the dominant term.
 #pragma once
 
 #include <cmath>
 
 #include "ptx.cuh"
 
+#include <cuda_fp16.h>
+
 namespace b2a {
 
 constexpr int kMergePairs = 256;     // (s, h) pairs per block = threads per block
 constexpr int kMergeMaxP = 64;       // shared weights: P x 256 floats
 
-template <int D>
+// Widens one 16-byte unit of partial values to fp32.
+template <typename T>
+__device__ __forceinline__ void unpack_unit(const uint4& x, float (&v)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 4) {
+    v[0] = __uint_as_float(x.x);
+    v[1] = __uint_as_float(x.y);
+    v[2] = __uint_as_float(x.z);
+    v[3] = __uint_as_float(x.w);
+  } else {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h;
+      memcpy(&h, &w[i], 4);
+      const float2 f = __half22float2(h);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+}
+
+// T: float (fp32 partials) or uint16_t (fp16 partials).
+template <int D, typename T>
 __global__ void __launch_bounds__(kMergePairs)
-    attn_merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ lse_parts, int P,
+    attn_merge_kernel(const T* __restrict__ o_parts, const float* __restrict__ lse_parts, int P,
                       int S, int H, uint16_t* __restrict__ out, float* __restrict__ lse_out) {
   extern __shared__ float w_s[];  // [P][kMergePairs]
   const long long npairs = static_cast<long long>(S) * H;
@@ -61,12 +87,13 @@ __global__ void __launch_bounds__(kMergePairs)
   }
   __syncthreads();
 
-  constexpr int U = D / 4;  // float4 units per pair
+  constexpr int E = 16 / static_cast<int>(sizeof(T));  // partial values per 16-byte unit
+  constexpr int U = D / E;                              // units per pair
   const long long pairs_here = (npairs - pair0 < kMergePairs) ? (npairs - pair0) : kMergePairs;
   const int units = static_cast<int>(pairs_here) * U;
-  const float4* src = reinterpret_cast<const float4*>(o_parts) + pair0 * U;
-  const size_t plane4 = static_cast<size_t>(npairs) * U;  // float4 per chunk
-  uint2* dst = reinterpret_cast<uint2*>(out) + pair0 * U;
+  const uint4* src = reinterpret_cast<const uint4*>(o_parts) + pair0 * U;
+  const size_t plane16 = static_cast<size_t>(npairs) * U;  // units per chunk
+  uint16_t* dst = out + pair0 * D;
 
   // Two units per thread per pass, all their chunk loads issued before use,
   // so each thread keeps up to 16 independent 16-byte loads in flight.
@@ -75,37 +102,46 @@ __global__ void __launch_bounds__(kMergePairs)
     const bool has1 = u1 < units;
     const int pi0 = u0 / U;
     const int pi1 = has1 ? u1 / U : pi0;
-    float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 acc1 = acc0;
+    float acc0[E], acc1[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc0[e] = acc1[e] = 0.f;
     for (int q0 = 0; q0 < P; q0 += 8) {
-      float4 x0[8], x1[8];
+      uint4 x0[8], x1[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (q0 + i < P) {
-          x0[i] = __ldcs(src + (q0 + i) * plane4 + u0);
-          if (has1) x1[i] = __ldcs(src + (q0 + i) * plane4 + u1);
+          x0[i] = __ldcs(src + (q0 + i) * plane16 + u0);
+          if (has1) x1[i] = __ldcs(src + (q0 + i) * plane16 + u1);
         }
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (q0 + i < P) {
+          float v[E];
           const float w0 = w_s[(q0 + i) * kMergePairs + pi0];
-          acc0.x = fmaf(w0, x0[i].x, acc0.x);
-          acc0.y = fmaf(w0, x0[i].y, acc0.y);
-          acc0.z = fmaf(w0, x0[i].z, acc0.z);
-          acc0.w = fmaf(w0, x0[i].w, acc0.w);
+          unpack_unit<T>(x0[i], v);
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc0[e] = fmaf(w0, v[e], acc0[e]);
           if (has1) {
             const float w1 = w_s[(q0 + i) * kMergePairs + pi1];
-            acc1.x = fmaf(w1, x1[i].x, acc1.x);
-            acc1.y = fmaf(w1, x1[i].y, acc1.y);
-            acc1.z = fmaf(w1, x1[i].z, acc1.z);
-            acc1.w = fmaf(w1, x1[i].w, acc1.w);
+            unpack_unit<T>(x1[i], v);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc1[e] = fmaf(w1, v[e], acc1[e]);
           }
         }
       }
     }
-    dst[u0] = make_uint2(pack_half2(acc0.x, acc0.y), pack_half2(acc0.z, acc0.w));
-    if (has1) dst[u1] = make_uint2(pack_half2(acc1.x, acc1.y), pack_half2(acc1.z, acc1.w));
+    if constexpr (E == 4) {
+      reinterpret_cast<uint2*>(dst)[u0] = make_uint2(pack_half2(acc0[0], acc0[1]), pack_half2(acc0[2], acc0[3]));
+      if (has1)
+        reinterpret_cast<uint2*>(dst)[u1] = make_uint2(pack_half2(acc1[0], acc1[1]), pack_half2(acc1[2], acc1[3]));
+    } else {
+      reinterpret_cast<uint4*>(dst)[u0] = make_uint4(pack_half2(acc0[0], acc0[1]), pack_half2(acc0[2], acc0[3]),
+                                                     pack_half2(acc0[4], acc0[5]), pack_half2(acc0[6], acc0[7]));
+      if (has1)
+        reinterpret_cast<uint4*>(dst)[u1] = make_uint4(pack_half2(acc1[0], acc1[1]), pack_half2(acc1[2], acc1[3]),
+                                                       pack_half2(acc1[4], acc1[5]), pack_half2(acc1[6], acc1[7]));
+    }
   }
 }
 

@@ -283,7 +283,7 @@ int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, f
   if (Skv == 0) {
     const size_t n_o = static_cast<size_t>(Sq) * H * d;
     const size_t n_l = static_cast<size_t>(Sq) * H;
-    b2a::attn_empty_partial_kernel<<<di->sm_count * 4, 256, 0, stream>>>(o_part, lse_part, n_o, n_l);
+    b2a::attn_empty_partial_kernel<float><<<di->sm_count * 4, 256, 0, stream>>>(o_part, lse_part, n_o, n_l);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? B2A_OK : cuda_fail(e);
   }
@@ -292,6 +292,33 @@ int attn_partial_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, f
   prm.lse_part = lse_part;
   prm.status = di->status;
   return launch_any<b2a::kModePartial>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
+}
+
+// FP16 split-reduction partial: the monolithic epilogue (o / l rounded to
+// fp16, lse in fp32) pointed at the chunk's [Sq, H, d] slot and [H, Sq] row.
+int attn_partial_f16_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o_part,
+                          float* lse_part, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_kv,
+                          cudaStream_t stream) {
+  int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_kv, ld_kv);
+  if (st != B2A_OK) return st;
+  if (!o_part || !lse_part || !aligned16(o_part) || (reinterpret_cast<uintptr_t>(lse_part) & 3u))
+    return B2A_ERR_INVALID_ARG;
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  if (Skv == 0) {
+    const size_t n_o = static_cast<size_t>(Sq) * H * d;
+    const size_t n_l = static_cast<size_t>(Sq) * H;
+    b2a::attn_empty_partial_kernel<uint16_t><<<di->sm_count * 4, 256, 0, stream>>>(o_part, lse_part, n_o, n_l);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+  }
+  b2a::AttnParams prm{};
+  prm.out = o_part;
+  prm.ld_o = H * d;
+  prm.lse = lse_part;
+  prm.lse_ld = Sq;
+  prm.status = di->status;
+  return launch_any<b2a::kModeFwd>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
 }
 
 int attn_accum_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_acc, float* lse_acc,
@@ -319,8 +346,9 @@ int attn_accum_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, flo
   return launch_any<b2a::kModeAccum>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
 }
 
-int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
-                    int S, int H, int d, cudaStream_t stream) {
+template <typename T>
+int launch_merge(const T* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S, int H,
+                 int d, cudaStream_t stream) {
   if (!o_parts || !lse_parts || !out) return B2A_ERR_INVALID_ARG;
   if (!aligned16(o_parts) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
     return B2A_ERR_INVALID_ARG;
@@ -334,20 +362,18 @@ int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_
   int st = current_device(&di);
   if (st != B2A_OK) return st;
   const int smem = P * b2a::kMergePairs * static_cast<int>(sizeof(float));
-  cudaError_t e;
-  if (d == 128) {
-    e = cudaFuncSetAttribute(b2a::attn_merge_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    b2a::attn_merge_kernel<128><<<static_cast<unsigned>(blocks), b2a::kMergePairs, smem, stream>>>(
-        o_parts, lse_parts, P, S, H, out, lse_out);
-  } else {
-    e = cudaFuncSetAttribute(b2a::attn_merge_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    b2a::attn_merge_kernel<64><<<static_cast<unsigned>(blocks), b2a::kMergePairs, smem, stream>>>(
-        o_parts, lse_parts, P, S, H, out, lse_out);
-  }
+  auto kern = d == 128 ? b2a::attn_merge_kernel<128, T> : b2a::attn_merge_kernel<64, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  kern<<<static_cast<unsigned>(blocks), b2a::kMergePairs, smem, stream>>>(o_parts, lse_parts, P, S, H, out,
+                                                                          lse_out);
   e = cudaGetLastError();
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+}
+
+int attn_merge_impl(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out,
+                    int S, int H, int d, cudaStream_t stream) {
+  return launch_merge<float>(o_parts, lse_parts, P, out, lse_out, S, H, d, stream);
 }
 
 // q/k RMSNorm epilogue parameters (null: plain projection).
@@ -535,6 +561,13 @@ int attn_fwd_partial(const uint16_t* q, const uint16_t* k_chunk, const uint16_t*
                            static_cast<cudaStream_t>(stream));
 }
 
+int attn_fwd_partial_f16(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk, uint16_t* o_part,
+                         float* lse_part, int Sq, int Skv, int H, int d, float scale, int ld_q, int ld_kv,
+                         void* stream) {
+  return attn_partial_f16_impl(q, k_chunk, v_chunk, o_part, lse_part, Sq, Skv, H, d, scale, ld_q, ld_kv,
+                               static_cast<cudaStream_t>(stream));
+}
+
 int attn_fwd_accumulate(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk, float* o_acc,
                         float* lse_acc, uint16_t* out, int Sq, int Skv, int H, int d, float scale, int ld_q,
                         int ld_kv, void* stream) {
@@ -556,6 +589,11 @@ int b2a_attn_kernel_for(int d, int Skv) { return use_pair(d, Skv) ? B2A_ATTN_KER
 int attn_merge(const float* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S,
                int H, int d, void* stream) {
   return attn_merge_impl(o_parts, lse_parts, P, out, lse_out, S, H, d, static_cast<cudaStream_t>(stream));
+}
+
+int attn_merge_f16(const uint16_t* o_parts, const float* lse_parts, int P, uint16_t* out, float* lse_out, int S,
+                   int H, int d, void* stream) {
+  return launch_merge<uint16_t>(o_parts, lse_parts, P, out, lse_out, S, H, d, static_cast<cudaStream_t>(stream));
 }
 
 int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, int M, int N, int K, void* stream) {
@@ -755,7 +793,7 @@ const char* b2a_status_string(int status) {
 
 int b2a_last_cuda_error(void) { return t_last_cuda_error; }
 
-int b2a_version(void) { return 101; }
+int b2a_version(void) { return 102; }
 
 #ifdef B2A_TRACE
 // Trace builds only: choose the traced CTA, then read the event table

@@ -74,6 +74,19 @@ def merge(o_parts, lse_parts):
     return o, lse
 
 
+def fp16_partials(o_parts):
+    """The FP16 split-reduction: partial outputs stored in fp16.
+
+    The accuracy table of "TensorRT Multi-Device (multi-GPU) support"
+    (Validation) attributes the multi-device error to an FP16 split-reduction.
+    Reading: each chunk's normalised output ``o_p`` is rounded to fp16
+    (round to nearest, ties to even) where it is stored, while ``lse_p`` stays
+    fp32; the merge above then runs on the rounded values.  numpy's float64 ->
+    float16 cast rounds once, to nearest even.  Returns float16 ``o_parts``.
+    """
+    return np.asarray(o_parts, dtype=np.float64).astype(np.float16)
+
+
 def accumulate(o_acc, lse_acc, o_c, lse_c):
     """One ring step: fold chunk ``(o_c, lse_c)`` into the running ``(o_acc, lse_acc)``.
 

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.b2a_version() == 101
+    assert lib.b2a_version() == 102
     assert lib.b2a_status_string(0) == b"ok"
     assert lib.b2a_status_string(1) == b"invalid argument"
     assert lib.b2a_status_string(4) == b"device-side wait timed out"
@@ -80,6 +80,23 @@ def test_partial_and_merge_reject(lib):
     assert m(FAKE, FAKE, 65, FAKE, None, 16, 2, 64, None) == 2    # P above the limit
     assert m(FAKE, FAKE, 2, FAKE, None, 16, 2, 80, None) == 1     # d
     assert m(FAKE + 4, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1  # alignment
+    assert m(None, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1
+
+
+def test_fp16_partial_and_merge_reject(lib):
+    p = lib.attn_fwd_partial_f16
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 64, 0.1, 128, 128, None) == 1   # Sq = 0
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, 4, -1, 2, 64, 0.1, 128, 128, None) == 1  # Skv < 0
+    assert p(FAKE, FAKE, FAKE, None, FAKE, 4, 4, 2, 64, 0.1, 128, 128, None) == 1   # o_part
+    assert p(FAKE, FAKE, FAKE, FAKE + 8, FAKE, 4, 4, 2, 64, 0.1, 128, 128, None) == 1
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 4, 2, 64, 0.1, 128, 128, None) == 1  # lse_part
+    assert p(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 2, 96, 0.1, 128, 128, None) == 1   # d
+    m = lib.attn_merge_f16
+    assert m(FAKE, FAKE, 0, FAKE, None, 16, 2, 64, None) == 1     # P = 0
+    assert m(FAKE, FAKE, 65, FAKE, None, 16, 2, 64, None) == 2    # P above the limit
+    assert m(FAKE, FAKE, 2, FAKE, None, 16, 2, 80, None) == 1     # d
+    assert m(FAKE + 8, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1  # alignment
+    assert m(FAKE, FAKE, 2, FAKE + 2, None, 16, 2, 64, None) == 1
     assert m(None, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1
 
 

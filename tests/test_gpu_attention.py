@@ -41,8 +41,8 @@ def run_mono(b2a, q, k, v, scale):
     return host(out).astype(np.float64), host(lse).astype(np.float64)
 
 
-def run_chunked(b2a, q, k, v, scale, P):
-    out, lse = b2a.attn_chunked(dev(q), dev(k), dev(v), P, scale=scale)
+def run_chunked(b2a, q, k, v, scale, P, partial_dtype=torch.float32):
+    out, lse = b2a.attn_chunked(dev(q), dev(k), dev(v), P, scale=scale, partial_dtype=partial_dtype)
     b2a.check_status()
     return host(out).astype(np.float64), host(lse).astype(np.float64)
 
@@ -170,6 +170,9 @@ def test_tiny_workload_full(b2a):
     out2, lse2 = run_chunked(b2a, q, k, v, w.scale, w.P)
     assert_out_close(out2, ref, "tiny chunked")
     assert_lse_close(lse2, ref_lse)
+    out3, lse3 = run_chunked(b2a, q, k, v, w.scale, w.P, torch.float16)
+    assert_out_close(out3, ref, "tiny chunked, fp16 partials")
+    assert_lse_close(lse3, ref_lse)
 
 
 def test_seq8k_workload_full(b2a):
@@ -182,6 +185,9 @@ def test_seq8k_workload_full(b2a):
     out2, lse2 = run_chunked(b2a, q, k, v, w.scale, w.P)
     assert_out_close(out2, ref, "8k chunked")
     assert_lse_close(lse2, ref_lse)
+    out3, lse3 = run_chunked(b2a, q, k, v, w.scale, w.P, torch.float16)
+    assert_out_close(out3, ref, "8k chunked, fp16 partials")
+    assert_lse_close(lse3, ref_lse)
 
 
 def _sampled_check(b2a, w, P):
@@ -207,6 +213,17 @@ def _sampled_check(b2a, w, P):
         # sharded vs unsharded on every element
         assert_out_close(o2h.astype(np.float64), out_h.astype(np.float64), f"{w.name} chunked vs mono")
         assert_lse_close(l2h, lse_h, f"{w.name} chunked vs mono lse")
+        del out2, lse2
+        # the FP16 split-reduction form
+        out3, lse3 = b2a.attn_chunked(qd, kd, vd, P, scale=w.scale, partial_dtype=torch.float16)
+        b2a.check_status()
+        o3h, l3h = host(out3), host(lse3)
+        got3 = np.stack([o3h[rows[h], h, :] for h in range(w.H)], axis=1).astype(np.float64)
+        got3_lse = np.stack([l3h[h, rows[h]] for h in range(w.H)]).astype(np.float64)
+        assert_out_close(got3, ref, f"{w.name} chunked fp16 partials sampled")
+        assert_lse_close(got3_lse, ref_lse)
+        assert_out_close(o3h.astype(np.float64), out_h.astype(np.float64), f"{w.name} fp16 partials vs mono")
+        assert_lse_close(l3h, lse_h, f"{w.name} fp16 partials vs mono lse")
 
 
 def test_seq32k_qsigma4_workload_sampled(b2a):

@@ -306,6 +306,45 @@ def test_ring_step_order_does_not_matter():
     np.testing.assert_allclose(fwd[1], lm, atol=1e-13)
 
 
+def test_fp16_partials_round_to_nearest_even():
+    # fp16 spacing at 1 is 2^-10: 1 + 2^-11 is a tie and goes to the even
+    # neighbour 1; 1 + 3*2^-11 ties between odd 1 + 2^-10 and even 1 + 2^-9;
+    # below 2^-14 the spacing is 2^-24 (subnormals)
+    got = C.fp16_partials(np.array([1 + 2 ** -11, 1 + 3 * 2 ** -11, -(1 + 2 ** -11), 3 * 2 ** -25, 0.1]))
+    assert got.dtype == np.float16
+    want = [1.0, 1 + 2 ** -9, -1.0, 2 ** -23, struct.unpack("<e", struct.pack("<e", 0.1))[0]]
+    assert [float(x) for x in got] == want
+
+
+def test_fp16_partials_single_chunk_is_the_rounded_output():
+    # one chunk has weight exactly 1: the merge returns the stored fp16 values
+    q, k, v = rand_qkv(7, 2, 8, seed=31, Skv=23, sigma=2.0)
+    o_parts, lse_parts = C.partials(q, k, v, 0.4, 1)
+    o16 = C.fp16_partials(o_parts)
+    om, lm = C.merge(o16, lse_parts)
+    np.testing.assert_array_equal(om, o16[0].astype(np.float64))
+    np.testing.assert_array_equal(lm, lse_parts[0])
+
+
+def test_fp16_partials_error_within_half_ulp_of_the_partials():
+    # the merge weights are >= 0 and sum to 1, so rounding each partial by at
+    # most half an fp16 ulp moves the merged value by at most the largest
+    # such half ulp among the chunks; the lse does not change at all
+    q, k, v = rand_qkv(40, 3, 16, seed=37, Skv=90, sigma=3.0)
+    o_parts, lse_parts = C.partials(q, k, v, 0.25, 6)
+    exact, lse_e = C.merge(o_parts, lse_parts)
+    o16 = C.fp16_partials(o_parts)
+    got, lse_g = C.merge(o16, lse_parts)
+    half_ulp = np.spacing(np.abs(o16).astype(np.float16)).astype(np.float64) / 2
+    bound = half_ulp.max(axis=0)
+    err = np.abs(got - exact)
+    assert np.all(err <= bound * (1 + 1e-9) + 1e-15)
+    assert err.max() > 0                       # the rounding did happen
+    np.testing.assert_array_equal(lse_g, lse_e)
+    # fp16-exact partials merge exactly as the fp64 merge does
+    np.testing.assert_array_equal(C.merge(o16.astype(np.float64), lse_parts)[0], got)
+
+
 # ----------------------------------------------------------------- stack ----
 
 def test_rmsnorm_closed_forms():
