@@ -264,6 +264,104 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row, int 
   }
 }
 
+// Named barriers over ``n`` threads (a multiple of 32): plain, and returning
+// the AND of every thread's ``v``.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// Epilogue of a 128-row tile in the monolithic and partial forms, staged
+// through shared memory.  The same values as attn_epilogue (O scaled by
+// 1/l in fp32, then fp16 or fp32), stored differently: each thread writes
+// its NC columns into ``stage`` ([128 rows x D] in the output type, 16-byte
+// chunks XOR-swizzled by row so that neither these writes nor the reads
+// below conflict on banks); after a barrier of the tile's 256 threads each
+// warp stores whole output rows, so a store instruction covers 256-512
+// contiguous bytes instead of 16 bytes in each of 32 rows.  ``stage`` must
+// be shared memory no MMA or copy touches any more.  All 256 threads call
+// this with the same ``ok``; with ok false nothing is written.
+template <int D, int MODE, int NC>
+__device__ __forceinline__ void attn_epilogue_staged(const AttnParams& p, int row0, int row_in_tile, int head,
+                                                     int col, bool write_lse, uint32_t tO, float m, float l,
+                                                     uint8_t* stage, int bar_id, int wt, int lane, bool ok) {
+  static_assert(MODE == kModeFwd || MODE == kModePartial, "accumulate mode reads o_acc: attn_epilogue");
+  static_assert(NC % 32 == 0, "whole 32-column TMEM loads");
+  constexpr int EB = MODE == kModeFwd ? 2 : 4;  // bytes per output element
+  constexpr int PITCH = D * EB;                 // staging bytes per row
+  constexpr int CHUNKS = PITCH / 16;            // 16-byte chunks per row
+  static_assert(CHUNKS >= 8, "the swizzle permutes 8 chunks");
+  if (!named_bar_and(bar_id, 256, ok)) return;
+  const float wc = 1.f / l;
+  const int sw = row_in_tile & 7;
+  uint8_t* srow = stage + row_in_tile * PITCH;
+#pragma unroll
+  for (int cb = 0; cb < NC; cb += 32) {
+    uint32_t o[32];
+    tmem_ld32(tO + cb, o);
+    tmem_wait_ld(o);
+    if constexpr (EB == 2) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = (col + cb) / 8 + i;
+        const uint32_t* a = o + 8 * i;
+        *reinterpret_cast<uint4*>(srow + ((c ^ sw) << 4)) =
+            make_uint4(pack_half2(__uint_as_float(a[0]) * wc, __uint_as_float(a[1]) * wc),
+                       pack_half2(__uint_as_float(a[2]) * wc, __uint_as_float(a[3]) * wc),
+                       pack_half2(__uint_as_float(a[4]) * wc, __uint_as_float(a[5]) * wc),
+                       pack_half2(__uint_as_float(a[6]) * wc, __uint_as_float(a[7]) * wc));
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = (col + cb) / 4 + i;
+        const uint32_t* a = o + 4 * i;
+        *reinterpret_cast<float4*>(srow + ((c ^ sw) << 4)) =
+            make_float4(__uint_as_float(a[0]) * wc, __uint_as_float(a[1]) * wc, __uint_as_float(a[2]) * wc,
+                        __uint_as_float(a[3]) * wc);
+      }
+    }
+  }
+  const int row = row0 + row_in_tile;
+  if (write_lse && row < p.Sq) {
+    const size_t li = static_cast<size_t>(head) * p.lse_ld + row;
+    const float lse2 = m + lg2_approx(l);
+    if constexpr (MODE == kModeFwd) {
+      if (p.lse) p.lse[li] = lse2 * kLn2;
+    } else {
+      p.lse_part[li] = lse2 * kLn2;
+    }
+  }
+  named_bar_sync(bar_id, 256);
+  uint8_t* dst;
+  size_t row_bytes;
+  if constexpr (MODE == kModeFwd) {
+    dst = reinterpret_cast<uint8_t*>(p.out) + static_cast<size_t>(head) * D * 2;
+    row_bytes = static_cast<size_t>(p.ld_o) * 2;
+  } else {
+    dst = reinterpret_cast<uint8_t*>(p.o_part) + static_cast<size_t>(head) * D * 4;
+    row_bytes = static_cast<size_t>(p.H) * D * 4;
+  }
+  const int rows = p.Sq - row0 < 128 ? p.Sq - row0 : 128;
+#pragma unroll 4
+  for (int i = wt * 32 + lane; i < rows * CHUNKS; i += 256) {
+    const int r = i / CHUNKS, c = i - r * CHUNKS;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + r * PITCH + ((c ^ (r & 7)) << 4));
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row0 + r) * row_bytes + (c << 4)) = v;
+  }
+}
+
 // Wait ignoring the abort flag, used only to drain in-flight async work.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
@@ -605,9 +703,21 @@ __global__ void __launch_bounds__(576, 1)
     l = lsum[row_in_tile];
 
     if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), (nkv - 1) & 1, abort_flag, p.status);
-    if (ok) {
+    if constexpr (MODE == kModeAccum) {
+      if (ok) {
+        tc_fence_after();
+        attn_epilogue<D, MODE, C::OH>(p, row, head, half * C::OH, half == 0, tO, m_used, l, la);
+      }
+    } else {
       tc_fence_after();
-      attn_epilogue<D, MODE, C::OH>(p, row, head, half * C::OH, half == 0, tO, m_used, l, la);
+      // Staging: query tile 0 over Q (its final o_done commit follows every
+      // QK), tile 1 over the K/V ring (its final o_done commit follows the
+      // kernel's last MMA, and every K/V load has been consumed by then).
+      uint8_t* stage = smem + (qt ? C::OFF_KV : C::OFF_Q);
+      static_assert(C::QT * C::Q_BYTES >= C::BM * D * 4 && C::STAGES * C::KV_BYTES >= C::BM * D * 4,
+                    "an fp32 output tile fits either staging area");
+      attn_epilogue_staged<D, MODE, C::OH>(p, q0 + qt * C::BM, row_in_tile, head, half * C::OH, half == 0, tO,
+                                           m_used, l, stage, 9 + qt, warp & 7, lane, ok);
     }
   }
 

@@ -82,6 +82,7 @@ struct AttnPairShape {
   static constexpr int THREADS = 384;
   static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_SYNC = 10, WARP_QK = 11;
   static constexpr int BAR_HANDOFF = 5;    // named barrier: MMA warp + helper warp
+  static constexpr int BAR_EPI = 6;        // named barrier: the 8 softmax warps (epilogue)
   static constexpr int P_ARRIVALS = 16;                        // 8 softmax warps x 2 CTAs
   static constexpr int ROWS_PER_PAIR = 2 * BM;
   __host__ __device__ static constexpr int tm_s(int buf) { return 128 * buf; }
@@ -443,9 +444,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     l = lsum[row_in_tile];
 
     if (ok) ok = mbar_wait_warp(bar(C::B_OF), 0, abort_flag, p.status);
-    if (ok) {
+    if constexpr (MODE == kModeAccum) {
+      if (ok) {
+        tc_fence_after();
+        attn_epilogue<D, MODE, C::HALF>(p, row, head, half * C::HALF, half == 0, tO, m_used, l, la);
+      }
+    } else {
       tc_fence_after();
-      attn_epilogue<D, MODE, C::HALF>(p, row, head, half * C::HALF, half == 0, tO, m_used, l, la);
+      // staged over this CTA's K/V ring: o_final follows the pair's last MMA,
+      // and every load into this CTA had landed before the MMAs that read it
+      static_assert(C::STAGES * C::STAGE_BYTES >= C::BM * D * 4, "an fp32 output tile fits the K/V ring");
+      attn_epilogue_staged<D, MODE, C::HALF>(p, q0, row_in_tile, head, half * C::HALF, half == 0, tO, m_used, l,
+                                             smem + C::OFF_KV, C::BAR_EPI, warp, lane, ok);
     }
   }
 
