@@ -183,87 +183,6 @@ __device__ __forceinline__ float accum_lse2(const AttnParams& p, int row, int he
   return -INFINITY;
 }
 
-// Epilogue of one softmax thread: its query row, NC output columns from
-// ``col`` (TMEM columns tO .. tO+NC-1 hold the un-normalised O), running
-// max ``m`` (log2 units), row sum ``l`` and, in accumulate mode, the row's
-// running lse ``la`` (log2 units).  Every lane runs the TMEM loads.
-template <int D, int MODE, int NC>
-__device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row, int head, int col, bool write_lse,
-                                              uint32_t tO, float m, float l, float la) {
-  static_assert(NC % 32 == 0, "whole 32-column TMEM loads");
-  const bool live = row < p.Sq;
-  const float lse2 = m + lg2_approx(l);  // this launch's keys, log2 units
-  float wc = 1.f / l;                    // weight of the TMEM accumulator
-  float wa = 0.f;                        // weight of the running output
-  float lse_new2 = lse2;
-  if constexpr (MODE == kModeAccum) {
-    if (la > -INFINITY) {
-      const float mx = fmaxf(la, lse2);
-      const float ea = ex2_approx(la - mx), ec = ex2_approx(lse2 - mx);
-      const float inv = 1.f / (ea + ec);
-      lse_new2 = mx + lg2_approx(ea + ec);
-      wa = ea * inv;
-      wc = ec * inv / l;
-    }
-  }
-#pragma unroll
-  for (int cb = 0; cb < NC; cb += 32) {
-    uint32_t o[32];
-    tmem_ld32(tO + cb, o);
-    tmem_wait_ld(o);
-    if (!live) continue;
-    const int c0 = col + cb;
-    if constexpr (MODE == kModeFwd) {
-      uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(row) * p.ld_o +
-                                            static_cast<size_t>(head) * D + c0);
-#pragma unroll
-      for (int c = 0; c < 32; c += 8)
-        dst[c >> 3] = make_uint4(pack_half2(__uint_as_float(o[c]) * wc, __uint_as_float(o[c + 1]) * wc),
-                                 pack_half2(__uint_as_float(o[c + 2]) * wc, __uint_as_float(o[c + 3]) * wc),
-                                 pack_half2(__uint_as_float(o[c + 4]) * wc, __uint_as_float(o[c + 5]) * wc),
-                                 pack_half2(__uint_as_float(o[c + 6]) * wc, __uint_as_float(o[c + 7]) * wc));
-    } else {
-      float4* acc = reinterpret_cast<float4*>(p.o_part + (static_cast<size_t>(row) * p.H + head) * D + c0);
-      float v[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(o[c]) * wc;
-      if constexpr (MODE == kModeAccum) {
-        if (wa > 0.f) {
-          float4 a[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) a[c] = acc[c];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            v[4 * c] = fmaf(wa, a[c].x, v[4 * c]);
-            v[4 * c + 1] = fmaf(wa, a[c].y, v[4 * c + 1]);
-            v[4 * c + 2] = fmaf(wa, a[c].z, v[4 * c + 2]);
-            v[4 * c + 3] = fmaf(wa, a[c].w, v[4 * c + 3]);
-          }
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-      if constexpr (MODE == kModeAccum) {
-        if (p.out) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (static_cast<size_t>(row) * p.H + head) * D + c0);
-#pragma unroll
-          for (int c = 0; c < 32; c += 8)
-            dst[c >> 3] = make_uint4(pack_half2(v[c], v[c + 1]), pack_half2(v[c + 2], v[c + 3]),
-                                     pack_half2(v[c + 4], v[c + 5]), pack_half2(v[c + 6], v[c + 7]));
-        }
-      }
-    }
-  }
-  if (live && write_lse) {
-    const size_t li = static_cast<size_t>(head) * p.lse_ld + row;
-    if constexpr (MODE == kModeFwd) {
-      if (p.lse) p.lse[li] = lse2 * kLn2;
-    } else {
-      p.lse_part[li] = lse_new2 * kLn2;
-    }
-  }
-}
-
 // Named barriers over ``n`` threads (a multiple of 32): plain, and returning
 // the AND of every thread's ``v``.
 __device__ __forceinline__ void named_bar_sync(int id, int n) {
@@ -282,28 +201,46 @@ __device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
   return r != 0;
 }
 
-// Epilogue of a 128-row tile in the monolithic and partial forms, staged
-// through shared memory.  The same values as attn_epilogue (O scaled by
-// 1/l in fp32, then fp16 or fp32), stored differently: each thread writes
-// its NC columns into ``stage`` ([128 rows x D] in the output type, 16-byte
-// chunks XOR-swizzled by row so that neither these writes nor the reads
-// below conflict on banks); after a barrier of the tile's 256 threads each
-// warp stores whole output rows, so a store instruction covers 256-512
-// contiguous bytes instead of 16 bytes in each of 32 rows.  ``stage`` must
-// be shared memory no MMA or copy touches any more.  All 256 threads call
+// Epilogue of a 128-row tile, staged through shared memory.  Values: O
+// scaled by 1/l in fp32, then fp16 (monolithic) or fp32 (partial); in
+// accumulate mode the merge wa * o_acc + wc * O with the row's running lse
+// (the exact log-sum-exp combine), optionally also rounded to fp16.  Each
+// thread writes its NC columns into ``stage`` ([128 rows x D] in the output
+// type, fp32 in accumulate mode; 16-byte chunks XOR-swizzled by row so that
+// neither these writes nor the reads below conflict on banks); after a
+// barrier of the tile's 256 threads each warp stores whole output rows, so
+// a store instruction covers 256-512 contiguous bytes instead of 16 bytes in
+// each of 32 rows (measured: 8-tile partial pass 662 -> 758 TFLOP/s).  ``stage`` must
+// be shared memory no MMA or copy touches any more; ``wa_s`` (accumulate
+// mode) 128 floats of free shared memory for the rows' o_acc weights; ``la``
+// the row's running lse (log2 units, accumulate mode).  All 256 threads call
 // this with the same ``ok``; with ok false nothing is written.
 template <int D, int MODE, int NC>
-__device__ __forceinline__ void attn_epilogue_staged(const AttnParams& p, int row0, int row_in_tile, int head,
+__device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row0, int row_in_tile, int head,
                                                      int col, bool write_lse, uint32_t tO, float m, float l,
-                                                     uint8_t* stage, int bar_id, int wt, int lane, bool ok) {
-  static_assert(MODE == kModeFwd || MODE == kModePartial, "accumulate mode reads o_acc: attn_epilogue");
+                                                     float la, uint8_t* stage, float* wa_s, int bar_id, int wt,
+                                                     int lane, bool ok) {
   static_assert(NC % 32 == 0, "whole 32-column TMEM loads");
-  constexpr int EB = MODE == kModeFwd ? 2 : 4;  // bytes per output element
+  constexpr int EB = MODE == kModeFwd ? 2 : 4;  // bytes per staged element
   constexpr int PITCH = D * EB;                 // staging bytes per row
   constexpr int CHUNKS = PITCH / 16;            // 16-byte chunks per row
   static_assert(CHUNKS >= 8, "the swizzle permutes 8 chunks");
   if (!named_bar_and(bar_id, 256, ok)) return;
-  const float wc = 1.f / l;
+  const float lse2 = m + lg2_approx(l);  // this launch's keys, log2 units
+  float wc = 1.f / l;                    // weight of the TMEM accumulator
+  float lse_new2 = lse2;
+  if constexpr (MODE == kModeAccum) {
+    float wa = 0.f;                      // weight of the running output
+    if (la > -INFINITY) {
+      const float mx = fmaxf(la, lse2);
+      const float ea = ex2_approx(la - mx), ec = ex2_approx(lse2 - mx);
+      const float inv = 1.f / (ea + ec);
+      lse_new2 = mx + lg2_approx(ea + ec);
+      wa = ea * inv;
+      wc = ec * inv / l;
+    }
+    if (write_lse) wa_s[row_in_tile] = wa;
+  }
   const int sw = row_in_tile & 7;
   uint8_t* srow = stage + row_in_tile * PITCH;
 #pragma unroll
@@ -336,11 +273,10 @@ __device__ __forceinline__ void attn_epilogue_staged(const AttnParams& p, int ro
   const int row = row0 + row_in_tile;
   if (write_lse && row < p.Sq) {
     const size_t li = static_cast<size_t>(head) * p.lse_ld + row;
-    const float lse2 = m + lg2_approx(l);
     if constexpr (MODE == kModeFwd) {
       if (p.lse) p.lse[li] = lse2 * kLn2;
     } else {
-      p.lse_part[li] = lse2 * kLn2;
+      p.lse_part[li] = lse_new2 * kLn2;
     }
   }
   named_bar_sync(bar_id, 256);
@@ -357,8 +293,27 @@ __device__ __forceinline__ void attn_epilogue_staged(const AttnParams& p, int ro
 #pragma unroll 4
   for (int i = wt * 32 + lane; i < rows * CHUNKS; i += 256) {
     const int r = i / CHUNKS, c = i - r * CHUNKS;
-    const uint4 v = *reinterpret_cast<const uint4*>(stage + r * PITCH + ((c ^ (r & 7)) << 4));
-    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(row0 + r) * row_bytes + (c << 4)) = v;
+    uint4 v = *reinterpret_cast<const uint4*>(stage + r * PITCH + ((c ^ (r & 7)) << 4));
+    uint8_t* g = dst + static_cast<size_t>(row0 + r) * row_bytes + (c << 4);
+    if constexpr (MODE == kModeAccum) {
+      float4 f = make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                             __uint_as_float(v.w));
+      const float wa = wa_s[r];
+      if (wa > 0.f) {
+        const float4 a = *reinterpret_cast<const float4*>(g);
+        f.x = fmaf(wa, a.x, f.x);
+        f.y = fmaf(wa, a.y, f.y);
+        f.z = fmaf(wa, a.z, f.z);
+        f.w = fmaf(wa, a.w, f.w);
+      }
+      *reinterpret_cast<float4*>(g) = f;
+      if (p.out) {
+        uint16_t* o16 = p.out + (static_cast<size_t>(row0 + r) * p.H + head) * D + 4 * c;
+        *reinterpret_cast<uint2*>(o16) = make_uint2(pack_half2(f.x, f.y), pack_half2(f.z, f.w));
+      }
+    } else {
+      *reinterpret_cast<uint4*>(g) = v;
+    }
   }
 }
 
@@ -703,12 +658,7 @@ __global__ void __launch_bounds__(576, 1)
     l = lsum[row_in_tile];
 
     if (ok) ok = mbar_wait_warp(bar(C::B_O + qt), (nkv - 1) & 1, abort_flag, p.status);
-    if constexpr (MODE == kModeAccum) {
-      if (ok) {
-        tc_fence_after();
-        attn_epilogue<D, MODE, C::OH>(p, row, head, half * C::OH, half == 0, tO, m_used, l, la);
-      }
-    } else {
+    {
       tc_fence_after();
       // Staging: query tile 0 over Q (its final o_done commit follows every
       // QK), tile 1 over the K/V ring (its final o_done commit follows the
@@ -716,8 +666,9 @@ __global__ void __launch_bounds__(576, 1)
       uint8_t* stage = smem + (qt ? C::OFF_KV : C::OFF_Q);
       static_assert(C::QT * C::Q_BYTES >= C::BM * D * 4 && C::STAGES * C::KV_BYTES >= C::BM * D * 4,
                     "an fp32 output tile fits either staging area");
-      attn_epilogue_staged<D, MODE, C::OH>(p, q0 + qt * C::BM, row_in_tile, head, half * C::OH, half == 0, tO,
-                                           m_used, l, stage, 9 + qt, warp & 7, lane, ok);
+      // the row-max exchange slots are free once both halves have read them
+      attn_epilogue<D, MODE, C::OH>(p, q0 + qt * C::BM, row_in_tile, head, half * C::OH, half == 0, tO,
+                                           m_used, l, la, stage, red, 9 + qt, warp & 7, lane, ok);
     }
   }
 

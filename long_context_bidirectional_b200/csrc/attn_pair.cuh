@@ -444,18 +444,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     l = lsum[row_in_tile];
 
     if (ok) ok = mbar_wait_warp(bar(C::B_OF), 0, abort_flag, p.status);
-    if constexpr (MODE == kModeAccum) {
-      if (ok) {
-        tc_fence_after();
-        attn_epilogue<D, MODE, C::HALF>(p, row, head, half * C::HALF, half == 0, tO, m_used, l, la);
-      }
-    } else {
+    {
       tc_fence_after();
       // staged over this CTA's K/V ring: o_final follows the pair's last MMA,
       // and every load into this CTA had landed before the MMAs that read it
       static_assert(C::STAGES * C::STAGE_BYTES >= C::BM * D * 4, "an fp32 output tile fits the K/V ring");
-      attn_epilogue_staged<D, MODE, C::HALF>(p, q0, row_in_tile, head, half * C::HALF, half == 0, tO, m_used, l,
-                                             smem + C::OFF_KV, C::BAR_EPI, warp, lane, ok);
+      // (the row-max exchange slots hold the rows' o_acc weights: both
+      // halves have read them)
+      attn_epilogue<D, MODE, C::HALF>(p, q0, row_in_tile, head, half * C::HALF, half == 0, tO, m_used, l,
+                                             la, smem + C::OFF_KV, red, C::BAR_EPI, warp, lane, ok);
     }
   }
 
