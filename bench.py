@@ -194,10 +194,13 @@ def committed_traffic(kernel: str, workload: str):
     ent = table.get(kernel, {}).get(workload)
     if not ent:
         return None
-    src = os.path.join(ROOT, "long_context_bidirectional_b200", "csrc", ent["source"])
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest()[:16] != ent["source_sha256_16"]:
-            return None
+    # the counters hold only while every source the kernel compiles from is unchanged
+    h = hashlib.sha256()
+    for name in ent["sources"]:
+        with open(os.path.join(ROOT, "long_context_bidirectional_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest()[:16] != ent["sources_sha256_16"]:
+        return None
     return ent["bytes_per_launch"]
 
 
