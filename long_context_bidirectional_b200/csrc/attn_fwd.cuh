@@ -57,6 +57,7 @@ struct AttnParams {
   float* o_part;      // partial: fp32 [Sq, H, D]; accumulate: running o_acc (in place)
   float* lse_part;    // partial: fp32 [H, Sq]; accumulate: running lse_acc (in place)
   unsigned int* status;
+  int wave;           // CTAs resident at once (one per SM); 0: no L2 prefetch of Q
 };
 
 template <int D>
@@ -430,6 +431,22 @@ __global__ void __launch_bounds__(576, 1)
             tma_load_3d(sKV + st * C::KV_BYTES + sb * C::SUB_BYTES, m, bar(C::B_KVF + st), sb * 64,
                         head, j * C::BN);
           ++issued;
+        }
+        if (j == 0 && p.wave > 0) {
+          // Q of the CTA that takes this SM about one wave later: start its
+          // DRAM read now so that CTA finds it in L2 (its K/V tiles are
+          // shared by the head's CTAs and usually there already).
+          const int next = blockIdx.y * gridDim.x + blockIdx.x + p.wave;
+          const int nx = next % gridDim.x, ny = next / gridDim.x;
+          if (ny < static_cast<int>(gridDim.y)) {
+#pragma unroll
+            for (int qt = 0; qt < C::QT; ++qt) {
+              const int row = nx * C::ROWS_PER_CTA + qt * C::BM;
+              if (row >= p.Sq) break;
+#pragma unroll
+              for (int sb = 0; sb < C::SUB; ++sb) tma_prefetch_l2_3d(&tm_q, sb * 64, ny, row);
+            }
+          }
         }
       }
       if (!ok) {

@@ -195,6 +195,9 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   auto kern = b2a::attn_fwd_kernel<D, MODE, B2A_ATTN_EMU>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  prm.wave = di->sm_count;  // shared memory and TMEM allow one CTA per SM
   dim3 grid((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, H);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
   e = cudaGetLastError();
