@@ -272,3 +272,16 @@ def test_host_entry_point_end_to_end(b2a, S):
     assert_out_close(outs[0].numpy().astype(np.float64), ref, "host back-to-back 1")
     assert_out_close(outs[1].numpy().astype(np.float64), ref2, "host back-to-back 2")
     assert_lse_close(lses[1].numpy(), ref2_lse)
+    # two streams, a workspace each, several rounds with no sync in between:
+    # the calls share the library's copy streams and overlap each other
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [torch.empty(b2a.host_workspace_bytes(S, H, d, P), dtype=torch.uint8, device="cuda") for P in (1, 4)]
+    for _ in range(3):
+        for i, P in enumerate((1, 4)):
+            b2a.attn_fwd_host(qhs[i], kh, vh, outs[i], lses[i], wss[i], P=P, scale=scale, stream=streams[i])
+    torch.cuda.synchronize()
+    b2a.check_status()
+    assert_out_close(outs[0].numpy().astype(np.float64), ref, "host two streams 1")
+    assert_lse_close(lses[0].numpy(), ref_lse)
+    assert_out_close(outs[1].numpy().astype(np.float64), ref2, "host two streams 2")
+    assert_lse_close(lses[1].numpy(), ref2_lse)
