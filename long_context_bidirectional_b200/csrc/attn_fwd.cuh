@@ -318,13 +318,6 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row0, int
   }
 }
 
-// Wait ignoring the abort flag, used only to drain in-flight async work.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return;
-  }
-}
 
 // 64-thread named barrier for the two warps that share rows (ids 1..8).
 __device__ __forceinline__ void pair_barrier(int id) {

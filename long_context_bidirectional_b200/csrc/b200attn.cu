@@ -39,6 +39,7 @@ struct DeviceInfo {
   bool supported = false;
   int sm_count = 0;
   unsigned int* status = nullptr;
+  mutable std::atomic<int> gemm_clusters{0};  // co-resident clusters of gemm_tn_kernel (0: not queried yet)
 };
 
 std::mutex g_dev_mu;
@@ -393,7 +394,7 @@ int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t*
   if (!aligned16(a) || !aligned16(w) || !aligned16(c) || (r && !aligned16(r))) return B2A_ERR_INVALID_ARG;
   if (M < 1 || N < 1 || K < 1 || (N % 8) != 0 || (K % 8) != 0) return B2A_ERR_INVALID_ARG;
   using G = b2a::GemmShape;
-  const long long tiles_m = (M + G::BM - 1) / G::BM;
+  const long long tiles_m = (M + G::PAIR_M - 1) / G::PAIR_M;  // 256 x 256 tiles, one per CTA pair
   const long long tiles_n = (N + G::BN - 1) / G::BN;
   if (tiles_m * tiles_n > INT_MAX) return B2A_ERR_UNSUPPORTED;
   const DeviceInfo* di = nullptr;
@@ -401,7 +402,7 @@ int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t*
   if (st != B2A_OK) return st;
   CUtensorMap ta, tb;
   if ((st = gemm_map(&ta, a, M, K, G::BM)) != B2A_OK) return st;
-  if ((st = gemm_map(&tb, w, N, K, G::BN)) != B2A_OK) return st;
+  if ((st = gemm_map(&tb, w, N, K, G::BN / 2)) != B2A_OK) return st;
   b2a::GemmParams prm{};
   prm.M = M;
   prm.N = N;
@@ -422,8 +423,24 @@ int gemm_impl(const uint16_t* a, const uint16_t* w, const uint16_t* r, uint16_t*
   auto kern = norm ? b2a::gemm_tn_kernel<true> : b2a::gemm_tn_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   if (e != cudaSuccess) return cuda_fail(e);
-  const int grid = prm.num_tiles < di->sm_count ? prm.num_tiles : di->sm_count;
-  kern<<<grid, G::THREADS, G::SMEM_BYTES, stream>>>(ta, tb, prm);
+  // persistent: as many clusters of two CTAs as run at once
+  int resident = di->gemm_clusters.load(std::memory_order_relaxed);
+  if (resident == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(di->sm_count & ~1), 1, 1);
+    cfg.blockDim = dim3(G::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = G::SMEM_BYTES;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n < 1) {
+      (void)cudaGetLastError();
+      n = di->sm_count / 2;
+    }
+    resident = n > 0 ? n : 1;
+    di->gemm_clusters.store(resident, std::memory_order_relaxed);
+  }
+  const int clusters = prm.num_tiles < resident ? prm.num_tiles : resident;
+  kern<<<dim3(2 * clusters, 1, 1), G::THREADS, G::SMEM_BYTES, stream>>>(ta, tb, prm);
   e = cudaGetLastError();
   return e == cudaSuccess ? B2A_OK : cuda_fail(e);
 }
