@@ -16,11 +16,12 @@
 // 256x256 output tile, 128 rows per CTA.  Every MMA is one M = 256
 // tcgen05.mma.cta_group::2 issued by the leader CTA: each CTA supplies its
 // 128 rows of A and half (128 rows) of W from its own shared memory and
-// keeps its 128 rows of the result in its own TMEM.  Per 64-wide K step each
-// SM loads 32 KB (A 16 KB + W half 16 KB) for 4 MMAs of 128 cycles, instead
-// of 48 KB for a 128x256 tile on one SM: the tensor core reads 64 instead of
-// 96 bytes of shared memory per clock and W's L2 traffic halves.
-// K in steps of 64 through a 6-stage TMA ring (128-byte swizzle); the loads
+// keeps its 128 rows of the result in its own TMEM.  Per 64 columns of K
+// each SM loads 32 KB (A 16 KB + W half 16 KB) for 4 MMAs of 128 cycles,
+// instead of 48 KB for a 128x256 tile on one SM: the tensor core reads 64
+// instead of 96 bytes of shared memory per clock and W's L2 traffic halves.
+// K in steps of 128 through a 3-stage TMA ring (two 128-byte-swizzled
+// blocks of 64 columns per operand and stage); the loads
 // of both CTAs complete on the leader's barriers.  Warp roles per CTA:
 //   warp 0     TMA producer (its CTA's A rows and W half)
 //   warp 1     TMEM allocator and (leader only) single-thread MMA issuer
@@ -52,11 +53,14 @@ struct GemmParams {
 };
 
 struct GemmShape {
-  static constexpr int BM = 128, BN = 256, BK = 64;  // per CTA: 128 rows; per pair: 256 x 256
+  static constexpr int BM = 128, BN = 256, BK = 128;  // per CTA: 128 rows; per pair: 256 x 256
   static constexpr int PAIR_M = 2 * BM;
-  static constexpr int STAGES = 6;
-  static constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-  static constexpr int B_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's half of the W tile
+  static constexpr int STAGES = 3;
+  static constexpr int KSUB = 64;                    // K columns per 128-byte swizzled block
+  static constexpr int A_SUB = BM * KSUB * 2;        // 16 KB: [128 rows x 128 B]
+  static constexpr int B_SUB = (BN / 2) * KSUB * 2;  // 16 KB
+  static constexpr int A_BYTES = BM * BK * 2;        // 32 KB
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;  // 32 KB: this CTA's half of the W tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
   // barriers: full[STAGES] (leader), empty[STAGES], acc_full[2],
@@ -74,6 +78,7 @@ struct GemmShape {
   static constexpr int ACCE_ARRIVALS = 8;            // 4 epilogue warps x 2 CTAs
   static constexpr int GROUP_M = 8;    // raster: 8 pair m-blocks share each n sweep
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory per CTA");
+  static_assert(A_SUB == B_SUB, "one K offset for both operands");
 };
 
 __device__ __forceinline__ void gemm_tile_coords(const GemmParams& p, int tile, int& mb, int& nb) {
@@ -254,8 +259,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           if (leader) mbar_arrive_expect_tx(bar(C::B_FULL + st), 2 * C::STAGE_BYTES);
           const uint32_t lf = map_to_rank(bar(C::B_FULL + st), 0);
           const uint32_t sa = sBase + st * C::STAGE_BYTES;
-          tma_load_2d_pair(sa, &tm_a, lf, kb * C::BK, arow);
-          tma_load_2d_pair(sa + C::A_BYTES, &tm_b, lf, kb * C::BK, brow);
+#pragma unroll
+          for (int sb = 0; sb < C::BK / C::KSUB; ++sb) {
+            tma_load_2d_pair(sa + sb * C::A_SUB, &tm_a, lf, kb * C::BK + sb * C::KSUB, arow);
+            tma_load_2d_pair(sa + C::A_BYTES + sb * C::B_SUB, &tm_b, lf, kb * C::BK + sb * C::KSUB, brow);
+          }
         }
       }
       st_cluster_u32(map_to_rank(smem_u32(const_cast<uint32_t*>(issued_by + rank)), 0),
@@ -281,8 +289,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const uint32_t sa = sBase + st * C::STAGE_BYTES;
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
-            mma_ss_pair(d_t, sw128_desc(sa + kk * 32, 16, 1024), sw128_desc(sa + C::A_BYTES + kk * 32, 16, 1024),
-                        idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            const uint32_t ko = (kk >> 2) * C::A_SUB + (kk & 3) * 32;   // A_SUB == B_SUB
+            mma_ss_pair(d_t, sw128_desc(sa + ko, 16, 1024), sw128_desc(sa + C::A_BYTES + ko, 16, 1024), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit_pair(bar(C::B_EMPTY + st));
         }
