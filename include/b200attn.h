@@ -386,7 +386,7 @@ B2A_API int b2a_last_cuda_error(void);
  * and those built on them) use for head dim 128.  The pages have no
  * counterpart; this is a tuning and testing control.
  *   B2A_ATTN_KERNEL_AUTO    (default) CTA pairs when the call has at least
- *                           96 key tiles of 128 (Skv > 12160), else single CTAs
+ *                           48 key tiles of 128 (Skv > 6016), else single CTAs
  *   B2A_ATTN_KERNEL_SINGLE  single CTAs, two 128-row query tiles each
  *   B2A_ATTN_KERNEL_PAIR    two-SM CTA pairs issuing M = 256 MMAs
  * Both compute the same result (the same arithmetic in the same order per

@@ -1,5 +1,5 @@
 // Non-causal attention forward on CTA pairs (sm_100a, head dim 128, calls
-// with at least 96 key tiles unless chosen explicitly).
+// with at least 48 key tiles unless chosen explicitly).
 //
 // Same result as attn_fwd_kernel, bit for bit (per head and query row: the softmax of the
 // scaled logits against every key, times V, and the natural-log LSE: "Multi-

@@ -210,9 +210,10 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
 // half of every K/V tile) when a launch has at least kPairMinKeyTiles key
 // tiles; shorter key ranges and head dim 64 run on single CTAs with two
 // query tiles, whose pipeline fills and drains in fewer SM-cycles per row
-// (measured on B200: the pair kernel is faster from 16384 keys up, the
-// single-CTA one at 8192 and below).
-constexpr int kPairMinKeyTiles = 96;
+// (measured on B200 with 32768 query rows: the pair kernel is faster from
+// 6144 keys up, by 0.5-1% there and 2-3% at 8192-12288, the single-CTA one by
+// 3% at 4096 keys).
+constexpr int kPairMinKeyTiles = 48;
 std::atomic<int> g_attn_kernel{B2A_ATTN_KERNEL_AUTO};
 
 bool use_pair(int d, int Skv) {
