@@ -234,8 +234,14 @@ def test_seq64k_workload_sampled(b2a):
     _sampled_check(b2a, W.SEQ64K, 1)
 
 
-def test_seq8k_h64_workload_sampled(b2a):
-    _sampled_check(b2a, W.SEQ8K_H64, 1)
+def test_seq8k_h64_workload_full(b2a):
+    # hidden 8192 (64 heads x 128) at S=8192: every row of every head
+    w = W.SEQ8K_H64
+    q, k, v = W.workload_qkv(w)
+    ref, ref_lse = OA.attention(q, k, v, w.scale)
+    out, lse = run_mono(b2a, q, k, v, w.scale)
+    assert_out_close(out, ref, "8k h64 mono")
+    assert_lse_close(lse, ref_lse)
 
 
 @pytest.mark.parametrize("S", [1000, 4500])
