@@ -2,8 +2,8 @@
 
 Default workload: S=32768, 32 heads x 128, Q ~ N(0, 4^2), K,V ~ N(0,1), fp16.
 One step = the whole hot path over that input: monolithic attention
-(attn_fwd) plus the ring-attention emulation (8 key-chunk partials with
-attn_fwd_partial, then attn_merge).  Both passes do 4*S^2*d*H flops, so the
+(attn_fwd) plus the ring-attention emulation (the 8 key-chunk partials with
+attn_fwd_partials, then attn_merge).  Both passes do 4*S^2*d*H flops, so the
 step's work is 2 * 4*S^2*d*H.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -273,9 +273,7 @@ def run_ours(args, rank, world, local):
         e0 = mark() if record else None
         b2a.attn_fwd(qd, kd, vd, out=out, lse=lse, scale=w.scale, stream=stream)
         e1 = mark() if record else None
-        for c, (lo, hi) in enumerate(bounds):
-            b2a.attn_fwd_partial(qd, kd[lo:hi], vd[lo:hi], o_parts[c], lse_parts[c], scale=w.scale,
-                                 stream=stream)
+        b2a.attn_fwd_partials(qd, kd, vd, P, o_parts, lse_parts, scale=w.scale, stream=stream)
         e2 = mark() if record else None
         b2a.attn_merge(o_parts, lse_parts, out=out_c, lse_out=lse_c, stream=stream)
         e3 = mark() if record else None
@@ -321,13 +319,20 @@ def run_ours(args, rank, world, local):
     # Roofline of each kernel of the step (per-launch averages from the CUDA
     # events above); the line's ``roofline`` is the one with the largest share.
     chunk_keys = max(hi_ - lo_ for lo_, hi_ in bounds)
+    # attn_fwd_partials: one launch of the single-CTA kernel over every chunk
+    # when the chunks are short enough for it (and none is empty)
+    part_kernel = attn_kernel_name(b2a, d, chunk_keys, 1)
+    one_launch = S >= P and part_kernel.startswith("attn_fwd_kernel")
+    part_launches = 1 if one_launch else P
     rl = [
         {"bound": "tensor", "kernel": attn_kernel_name(b2a, d, S, 0), "role": "attn_fwd (monolithic)",
          "launches_per_step": 1, "ms_per_launch": mono_ms, "achieved": mono_tflops, "unit": "TFLOP/s",
          "peak": pk["tc_burst"], "algorithmic": "4*S^2*d*H flops per launch"},
-        {"bound": "tensor", "kernel": attn_kernel_name(b2a, d, chunk_keys, 1), "role": "attn_fwd_partial",
-         "launches_per_step": P, "ms_per_launch": part_ms / P, "achieved": part_tflops, "unit": "TFLOP/s",
-         "peak": pk["tc_burst"], "algorithmic": "4*S*(S/P)*d*H flops per launch"},
+        {"bound": "tensor", "kernel": part_kernel, "role": f"attn_fwd_partials ({P} chunks)",
+         "launches_per_step": part_launches, "ms_per_launch": part_ms / part_launches, "achieved": part_tflops,
+         "unit": "TFLOP/s", "peak": pk["tc_burst"],
+         "algorithmic": ("4*S^2*d*H flops per launch (all chunks)" if one_launch
+                         else "4*S*(S/P)*d*H flops per launch (one chunk)")},
         {"bound": "hbm", "kernel": f"attn_merge_kernel<{d}, float>", "role": "attn_merge",
          "launches_per_step": 1, "ms_per_launch": merge_ms, "achieved": merge_gbs, "unit": "GB/s",
          "peak": pk["hbm_gbs"],
@@ -399,14 +404,22 @@ def run_ours(args, rank, world, local):
                                              scale=w.scale, stream=stream))
     del cp_out
 
+    # The same partials as one attn_fwd_partial call per chunk (what a ring
+    # rank does as each K/V block arrives).  Not part of ``value``.
+    def per_chunk_pass():
+        for c, (c_lo, c_hi) in enumerate(bounds):
+            b2a.attn_fwd_partial(qd, kd[c_lo:c_hi], vd[c_lo:c_hi], o_parts[c], lse_parts[c], scale=w.scale,
+                                 stream=stream)
+
+    pcc_ms = time_calls(per_chunk_pass, n=3)
+
     # The FP16 split-reduction: the same P partials stored in fp16, and the
     # merge reading them (half the partial bytes).  Not part of ``value``.
     o16_parts = torch.empty((P, S, H, d), dtype=torch.float16, device=dev)
 
     def part16_pass():
-        for c, (c_lo, c_hi) in enumerate(bounds):
-            b2a.attn_fwd_partial_f16(qd, kd[c_lo:c_hi], vd[c_lo:c_hi], o16_parts[c], lse_parts[c],
-                                     scale=w.scale, stream=stream)
+        b2a.attn_fwd_partials(qd, kd, vd, P, o16_parts, lse_parts, scale=w.scale, stream=stream,
+                              partial_dtype=torch.float16)
 
     p16_ms = time_calls(part16_pass, n=3)
     m16_ms = time_calls(lambda: b2a.attn_merge_f16(o16_parts, lse_parts, out=out_c, lse_out=lse_c,
@@ -473,7 +486,7 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
         "config": {"workload": w.name, "S": S, "H": H, "d": d, "P": P, "batch": 1,
                    "q_sigma": w.q_sigma, "kv_sigma": w.kv_sigma,
-                   "step": f"attn_fwd + {P} x attn_fwd_partial + attn_merge",
+                   "step": f"attn_fwd + attn_fwd_partials ({P} chunks) + attn_merge",
                    "step_flops": step_flops, "attn_kernel": args.attn_kernel,
                    "l2": f"inputs larger than L2 (Q,K,V {3 * S * H * d * 2 / 2**20:.0f} MiB, "
                          f"partials {P * S * H * d * 4 / 2**20:.0f} MiB per step)",
@@ -484,6 +497,9 @@ def run_ours(args, rank, world, local):
         "kernels": {"attn_fwd_ms": mono_ms, "attn_fwd_tflops": mono_tflops,
                     "partial_pass_ms": part_ms,
                     "partial_pass_tflops": part_tflops,
+                    "partial_pass": f"attn_fwd_partials, {P} chunks, {part_launches} launch(es) of {part_kernel}",
+                    "partial_per_chunk_calls_ms": pcc_ms,
+                    "partial_per_chunk_calls_tflops": w.flops / (pcc_ms * 1e-3) / 1e12,
                     "merge_ms": merge_ms, "merge_gbs": merge_gbs,
                     "ring_pass_ms": ring_ms,
                     "ring_pass_tflops": w.flops / (ring_ms * 1e-3) / 1e12,
@@ -499,10 +515,10 @@ def run_ours(args, rank, world, local):
                     "fp16_partial_pass_tflops": w.flops / (p16_ms * 1e-3) / 1e12,
                     "merge_f16_ms": m16_ms, "merge_f16_gbs": merge16_gbs,
                     "merge_f16_hbm_frac": merge16_gbs / pk["hbm_gbs"], "merge_f16_bytes": merge16_bytes,
-                    "fp16_split_reduction": f"{P} x attn_fwd_partial_f16 + attn_merge_f16 (not in value)"},
+                    "fp16_split_reduction": "attn_fwd_partials_f16 + attn_merge_f16 (not in value)"},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": args.steps * (P + 2),
+        "gpu_launches": args.steps * (part_launches + 2),
         "clocks": clocks,
     }
     if rank == 0:

@@ -147,6 +147,33 @@ B2A_API int attn_fwd_partial_f16(const uint16_t* q, const uint16_t* k_chunk, con
                                  int ld_q, int ld_kv, void* stream);
 
 /*
+ * attn_fwd_partials -- every key chunk's partial in one call: for c < P,
+ * chunk c = keys [floor(c*Skv/P), floor((c+1)*Skv/P)) of k, v, and
+ * (o_parts[c], lse_parts[c]) is what attn_fwd_partial returns for that
+ * chunk (the one-device form of ring attention's per-chunk partials, TensorRT
+ * 11.0 multi-device article, Ring Attention), bit for bit.  Chunks short
+ * enough for the single-CTA kernel (see b2a_set_attn_kernel) run as one
+ * launch over (row block, chunk, head), the chunk varying fastest so that
+ * the CTAs running at once share their Q tiles and K/V in L2; longer chunks
+ * run one CTA-pair launch each.
+ *
+ * q          device fp16 [Sq, H, d], row stride ld_q.
+ * k, v       device fp16 [Skv, H, d], row stride ld_kv (all keys).
+ * o_parts    device fp32 [P, Sq, H, d] contiguous, 16-byte aligned.
+ * lse_parts  device fp32 [P, H, Sq] contiguous.
+ * P >= 1; Skv >= 0 (empty chunks give o = 0, lse = -inf); other
+ * requirements and errors as attn_fwd_partial.
+ */
+B2A_API int attn_fwd_partials(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_parts,
+                              float* lse_parts, int Sq, int Skv, int P, int H, int d, float scale, int ld_q,
+                              int ld_kv, void* stream);
+
+/* attn_fwd_partials with fp16 o_parts ([P, Sq, H, d]; attn_fwd_partial_f16 per chunk). */
+B2A_API int attn_fwd_partials_f16(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o_parts,
+                                  float* lse_parts, int Sq, int Skv, int P, int H, int d, float scale, int ld_q,
+                                  int ld_kv, void* stream);
+
+/*
  * attn_fwd_accumulate -- one ring-attention step in place: fold the keys of
  * one chunk into a running result, the way each rank of ring attention
  * updates its output as K/V blocks arrive (TensorRT 11.0 multi-device

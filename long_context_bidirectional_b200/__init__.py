@@ -23,7 +23,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "lib
 
 __all__ = [
     "B2AError", "lib", "attn_fwd", "attn_fwd_batched", "attn_fwd_gathered_kv", "attn_fwd_partial", "attn_fwd_accumulate",
-    "attn_fwd_partial_f16", "attn_merge", "attn_merge_f16", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
+    "attn_fwd_partial_f16", "attn_fwd_partials", "attn_merge", "attn_merge_f16", "attn_chunked", "attn_ring", "set_attn_kernel", "get_attn_kernel", "attn_kernel_for",
     "ATTN_KERNEL_AUTO", "ATTN_KERNEL_SINGLE", "ATTN_KERNEL_PAIR",
     "qkv_proj", "qkv_proj_qknorm", "out_proj", "attn_block_fwd", "stack_forward", "attn_fwd_host",
     "host_workspace_bytes", "check_status", "selftest_wait_timeout",
@@ -50,6 +50,8 @@ _SIGS = {
     "attn_merge": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
     "attn_fwd_partial_f16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "attn_merge_f16": (_i, [_vp, _vp, _i, _vp, _vp, _i, _i, _i, _vp]),
+    "attn_fwd_partials": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
+    "attn_fwd_partials_f16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _f, _i, _i, _vp]),
     "qkv_proj": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp]),
     "attn_block_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
     "attn_block_fwd_static": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _f, _vp]),
@@ -215,6 +217,37 @@ def attn_fwd_partial_f16(q, k_chunk, v_chunk, o_part=None, lse_part=None, scale=
     return _partial("attn_fwd_partial_f16", torch.float16, q, k_chunk, v_chunk, o_part, lse_part, scale, stream)
 
 
+def attn_fwd_partials(q, k, v, P: int, o_parts=None, lse_parts=None, scale=None, stream=None,
+                      partial_dtype=torch.float32):
+    """Every key chunk's partial in one call: ``(o_parts [P,Sq,H,d], lse_parts [P,H,Sq])``,
+    chunk c = keys ``chunk_bounds(Skv, P)[c]`` (fp32 or fp16 ``o_parts``)."""
+    Sq, H, d = q.shape
+    ld_q = _check_qkv("q", q)
+    Skv = k.shape[0]
+    ld_k = _check_qkv("k", k, H, d)
+    ld_v = _check_qkv("v", v, H, d)
+    if v.shape[0] != Skv:
+        raise ValueError("k and v need the same length")
+    if ld_k != ld_v:
+        raise ValueError("k and v must share a row stride")
+    if partial_dtype not in (torch.float32, torch.float16):
+        raise ValueError("partial_dtype must be torch.float32 or torch.float16")
+    if o_parts is None:
+        o_parts = torch.empty((P, Sq, H, d), dtype=partial_dtype, device=q.device)
+    if lse_parts is None:
+        lse_parts = torch.empty((P, H, Sq), dtype=torch.float32, device=q.device)
+    if not (o_parts.is_contiguous() and o_parts.dtype == partial_dtype and o_parts.numel() == P * Sq * H * d):
+        raise ValueError(f"o_parts must be contiguous {partial_dtype} [P, Sq, H, d]")
+    if not (lse_parts.is_contiguous() and lse_parts.dtype == torch.float32 and lse_parts.numel() == P * H * Sq):
+        raise ValueError("lse_parts must be contiguous float32 [P, H, Sq]")
+    fn = "attn_fwd_partials_f16" if partial_dtype == torch.float16 else "attn_fwd_partials"
+    kp = k.data_ptr() if Skv > 0 else q.data_ptr()
+    vp = v.data_ptr() if Skv > 0 else q.data_ptr()
+    _call(fn, q.data_ptr(), kp, vp, o_parts.data_ptr(), lse_parts.data_ptr(), Sq, Skv, int(P), H, d,
+          _default_scale(d, scale), ld_q, ld_k if Skv > 0 else ld_q, _stream(stream))
+    return o_parts, lse_parts
+
+
 def _partial(fn, odt, q, k_chunk, v_chunk, o_part, lse_part, scale, stream):
     Sq, H, d = q.shape
     ld_q = _check_qkv("q", q)
@@ -353,9 +386,7 @@ def attn_chunked(q, k, v, P: int, out=None, lse=None, scale=None, o_parts=None, 
         o_parts = torch.empty((P, S, H, d), dtype=partial_dtype, device=q.device)
     if lse_parts is None:
         lse_parts = torch.empty((P, H, S), dtype=torch.float32, device=q.device)
-    part = attn_fwd_partial_f16 if f16 else attn_fwd_partial
-    for c, (lo, hi) in enumerate(chunk_bounds(k.shape[0], P)):
-        part(q, k[lo:hi], v[lo:hi], o_parts[c], lse_parts[c], scale=scale, stream=stream)
+    attn_fwd_partials(q, k, v, P, o_parts, lse_parts, scale=scale, stream=stream, partial_dtype=partial_dtype)
     merge = attn_merge_f16 if f16 else attn_merge
     return merge(o_parts, lse_parts, out=out, lse_out=lse, stream=stream)
 

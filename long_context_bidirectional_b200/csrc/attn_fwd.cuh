@@ -58,6 +58,13 @@ struct AttnParams {
   float* lse_part;    // partial: fp32 [H, Sq]; accumulate: running lse_acc (in place)
   unsigned int* status;
   int wave;           // CTAs resident at once (one per SM); 0: no L2 prefetch of Q
+  // Key chunks in one launch (single-CTA kernel): with nchunks = P > 1, chunk
+  // c = keys [c*Skv/P, (c+1)*Skv/P) and its outputs sit at out / o_part +
+  // c * out_chunk_stride and lse / lse_part + c * lse_chunk_stride
+  // (elements); grid.x = row blocks * P with the chunk varying fastest.
+  int nchunks;
+  long long out_chunk_stride;
+  long long lse_chunk_stride;
 };
 
 template <int D>
@@ -232,6 +239,8 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row0, int
   constexpr int CHUNKS = PITCH / 16;            // 16-byte chunks per row
   static_assert(CHUNKS >= 8, "the swizzle permutes 8 chunks");
   if (!named_bar_and(bar_id, 256, ok)) return;
+  // this CTA's key chunk (0 unless one launch covers several)
+  const size_t chunk = p.nchunks > 1 ? static_cast<size_t>(blockIdx.x % p.nchunks) : 0;
   const float lse2 = m + lg2_approx(l);  // this launch's keys, log2 units
   float wc = 1.f / l;                    // weight of the TMEM accumulator
   float lse_new2 = lse2;
@@ -278,7 +287,7 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row0, int
   }
   const int row = row0 + row_in_tile;
   if (write_lse && row < p.Sq) {
-    const size_t li = static_cast<size_t>(head) * p.lse_ld + row;
+    const size_t li = chunk * p.lse_chunk_stride + static_cast<size_t>(head) * p.lse_ld + row;
     if constexpr (MODE == kModeFwd) {
       if (p.lse) p.lse[li] = lse2 * kLn2;
     } else {
@@ -289,10 +298,10 @@ __device__ __forceinline__ void attn_epilogue(const AttnParams& p, int row0, int
   uint8_t* dst;
   size_t row_bytes;
   if constexpr (MODE == kModeFwd) {
-    dst = reinterpret_cast<uint8_t*>(p.out) + static_cast<size_t>(head) * D * 2;
+    dst = reinterpret_cast<uint8_t*>(p.out + chunk * p.out_chunk_stride) + static_cast<size_t>(head) * D * 2;
     row_bytes = static_cast<size_t>(p.ld_o) * 2;
   } else {
-    dst = reinterpret_cast<uint8_t*>(p.o_part) + static_cast<size_t>(head) * D * 4;
+    dst = reinterpret_cast<uint8_t*>(p.o_part + chunk * p.out_chunk_stride) + static_cast<size_t>(head) * D * 4;
     row_bytes = static_cast<size_t>(p.H) * D * 4;
   }
   const int rows = p.Sq - row0 < 128 ? p.Sq - row0 : 128;
@@ -358,8 +367,15 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
-  const int q0 = blockIdx.x * C::ROWS_PER_CTA;
-  const int nkv = (p.Skv + C::BN - 1) / C::BN;
+  // key chunk of this CTA (the whole key range unless the launch covers
+  // several chunks; then the chunk varies fastest, so the CTAs running at
+  // once share their Q tiles and the head's K/V in L2)
+  const int nch = p.nchunks > 1 ? p.nchunks : 1;
+  const int chunk = static_cast<int>(blockIdx.x) % nch;
+  const int q0 = (static_cast<int>(blockIdx.x) / nch) * C::ROWS_PER_CTA;
+  const int key0 = static_cast<int>(static_cast<long long>(chunk) * p.Skv / nch);
+  const int klen = static_cast<int>(static_cast<long long>(chunk + 1) * p.Skv / nch) - key0;
+  const int nkv = (klen + C::BN - 1) / C::BN;  // >= 1: the host never launches an empty chunk
 #ifdef B2A_TRACE
   const bool tracing = blockIdx.x == g_attn_trace_cta[0] && blockIdx.y == g_attn_trace_cta[1];
 #endif
@@ -427,7 +443,7 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
           for (int sb = 0; sb < C::SUB; ++sb)
             tma_load_3d(sKV + st * C::KV_BYTES + sb * C::SUB_BYTES, m, bar(C::B_KVF + st), sb * 64,
-                        head, j * C::BN);
+                        head, key0 + j * C::BN);
           ++issued;
         }
         if (j == 0 && p.wave > 0) {
@@ -435,7 +451,7 @@ __global__ void __launch_bounds__(576, 1)
           // DRAM read now so that CTA finds it in L2 (its K/V tiles are
           // shared by the head's CTAs and usually there already).
           const int next = blockIdx.y * gridDim.x + blockIdx.x + p.wave;
-          const int nx = next % gridDim.x, ny = next / gridDim.x;
+          const int nx = (next % gridDim.x) / nch, ny = next / gridDim.x;
           if (ny < static_cast<int>(gridDim.y)) {
 #pragma unroll
             for (int qt = 0; qt < C::QT; ++qt) {
@@ -571,11 +587,18 @@ __global__ void __launch_bounds__(576, 1)
         s[c] = __uint_as_float(r0[c]);
         s[32 + c] = __uint_as_float(r1[c]);
       }
-      const int valid = p.Skv - j * C::BN - half * C::HALF;
-      if (valid < C::HALF) {
+      if (j + 1 == nkv) {
+        // the chunk's last tile: keys past its end are masked (the key count
+        // is recomputed here rather than kept live through the loop)
+        const int ch = static_cast<int>(blockIdx.x) % nch;
+        const int kl = static_cast<int>(static_cast<long long>(ch + 1) * p.Skv / nch) -
+                       static_cast<int>(static_cast<long long>(ch) * p.Skv / nch);
+        const int valid = kl - j * C::BN - half * C::HALF;
+        if (valid < C::HALF) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= valid) s[c] = -INFINITY;
+          for (int c = 0; c < 64; ++c)
+            if (c >= valid) s[c] = -INFINITY;
+        }
       }
       // this half's row max: four independent 3-input max chains
       float ma = s[0], mb = s[1], mc = s[2], md = s[3];

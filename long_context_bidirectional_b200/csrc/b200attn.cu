@@ -199,7 +199,11 @@ int launch_attn(const void* q, const void* k, const void* v, int Sq, int Skv, in
   const DeviceInfo* di = nullptr;
   if ((st = current_device(&di)) != B2A_OK) return st;
   prm.wave = di->sm_count;  // shared memory and TMEM allow one CTA per SM
-  dim3 grid((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA, H);
+  // one CTA per (row block, key chunk), the chunk varying fastest
+  const long long gx = static_cast<long long>((Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA) *
+                       (prm.nchunks > 1 ? prm.nchunks : 1);
+  if (gx > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  dim3 grid(static_cast<unsigned>(gx), H);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
@@ -324,6 +328,58 @@ int attn_partial_f16_impl(const uint16_t* q, const uint16_t* k, const uint16_t* 
   prm.lse_ld = Sq;
   prm.status = di->status;
   return launch_any<b2a::kModeFwd>(q, k, v, Sq, Skv, H, d, ld_q, ld_kv, ld_kv, scale, prm, stream);
+}
+
+// All P key chunks' partials of one call (chunk c = keys [c*Skv/P,
+// (c+1)*Skv/P)): one launch of the single-CTA kernel over (row block, chunk,
+// head) when the chunks are short enough for it, else one CTA-pair launch
+// per chunk.  Per row the arithmetic is that of one attn_fwd_partial call
+// per chunk.
+int attn_partials_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, void* o_parts, float* lse_parts,
+                       int Sq, int Skv, int P, int H, int d, float scale, int ld_q, int ld_kv, bool f16,
+                       cudaStream_t stream) {
+  if (P < 1) return B2A_ERR_INVALID_ARG;
+  int st = validate_attn(q, k, v, Sq, Skv, H, d, scale, ld_q, ld_kv, ld_kv);
+  if (st != B2A_OK) return st;
+  if (!o_parts || !lse_parts || !aligned16(o_parts) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u))
+    return B2A_ERR_INVALID_ARG;
+  const size_t plane = static_cast<size_t>(Sq) * H * d;  // elements of one chunk's o_part
+  const size_t lplane = static_cast<size_t>(Sq) * H;
+  const int longest = static_cast<int>((static_cast<long long>(Skv) + P - 1) / P);
+  // every chunk has keys when Skv >= P (the kernel does not handle empty chunks)
+  if (Skv < P || use_pair(d, longest)) {
+    for (int c = 0; c < P; ++c) {
+      const long long lo = static_cast<long long>(c) * Skv / P;
+      const long long hi = static_cast<long long>(c + 1) * Skv / P;
+      const size_t off = static_cast<size_t>(lo) * ld_kv;
+      const int n = static_cast<int>(hi - lo);
+      st = f16 ? attn_partial_f16_impl(q, k + off, v + off, static_cast<uint16_t*>(o_parts) + c * plane,
+                                       lse_parts + c * lplane, Sq, n, H, d, scale, ld_q, ld_kv, stream)
+               : attn_partial_impl(q, k + off, v + off, static_cast<float*>(o_parts) + c * plane,
+                                   lse_parts + c * lplane, Sq, n, H, d, scale, ld_q, ld_kv, stream);
+      if (st != B2A_OK) return st;
+    }
+    return B2A_OK;
+  }
+  const DeviceInfo* di = nullptr;
+  if ((st = current_device(&di)) != B2A_OK) return st;
+  b2a::AttnParams prm{};
+  prm.status = di->status;
+  prm.nchunks = P;
+  prm.out_chunk_stride = static_cast<long long>(plane);
+  prm.lse_chunk_stride = static_cast<long long>(lplane);
+  prm.lse_ld = Sq;
+  if (f16) {
+    prm.out = static_cast<uint16_t*>(o_parts);
+    prm.ld_o = H * d;
+    prm.lse = lse_parts;
+    return d == 128 ? launch_attn<128, b2a::kModeFwd>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream)
+                    : launch_attn<64, b2a::kModeFwd>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
+  }
+  prm.o_part = static_cast<float*>(o_parts);
+  prm.lse_part = lse_parts;
+  return d == 128 ? launch_attn<128, b2a::kModePartial>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream)
+                  : launch_attn<64, b2a::kModePartial>(q, k, v, Sq, Skv, H, ld_q, ld_kv, ld_kv, scale, prm, stream);
 }
 
 int attn_accum_impl(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_acc, float* lse_acc,
@@ -589,6 +645,19 @@ int attn_fwd_partial_f16(const uint16_t* q, const uint16_t* k_chunk, const uint1
                                static_cast<cudaStream_t>(stream));
 }
 
+int attn_fwd_partials(const uint16_t* q, const uint16_t* k, const uint16_t* v, float* o_parts, float* lse_parts,
+                      int Sq, int Skv, int P, int H, int d, float scale, int ld_q, int ld_kv, void* stream) {
+  return attn_partials_impl(q, k, v, o_parts, lse_parts, Sq, Skv, P, H, d, scale, ld_q, ld_kv, false,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_partials_f16(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* o_parts,
+                          float* lse_parts, int Sq, int Skv, int P, int H, int d, float scale, int ld_q, int ld_kv,
+                          void* stream) {
+  return attn_partials_impl(q, k, v, o_parts, lse_parts, Sq, Skv, P, H, d, scale, ld_q, ld_kv, true,
+                            static_cast<cudaStream_t>(stream));
+}
+
 int attn_fwd_accumulate(const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk, float* o_acc,
                         float* lse_acc, uint16_t* out, int Sq, int Skv, int H, int d, float scale, int ld_q,
                         int ld_kv, void* stream) {
@@ -814,7 +883,7 @@ const char* b2a_status_string(int status) {
 
 int b2a_last_cuda_error(void) { return t_last_cuda_error; }
 
-int b2a_version(void) { return 102; }
+int b2a_version(void) { return 103; }
 
 #ifdef B2A_TRACE
 // Trace builds only: choose the traced CTA, then read the event table

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.b2a_version() == 102
+    assert lib.b2a_version() == 103
     assert lib.b2a_status_string(0) == b"ok"
     assert lib.b2a_status_string(1) == b"invalid argument"
     assert lib.b2a_status_string(4) == b"device-side wait timed out"
@@ -98,6 +98,18 @@ def test_fp16_partial_and_merge_reject(lib):
     assert m(FAKE + 8, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1  # alignment
     assert m(FAKE, FAKE, 2, FAKE + 2, None, 16, 2, 64, None) == 1
     assert m(None, FAKE, 2, FAKE, None, 16, 2, 64, None) == 1
+
+
+def test_partials_reject(lib):
+    for f in (lib.attn_fwd_partials, lib.attn_fwd_partials_f16):
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 0, 2, 64, 0.1, 128, 128, None) == 1     # P = 0
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 2, 2, 64, 0.1, 128, 128, None) == 1     # Sq = 0
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, -1, 2, 2, 64, 0.1, 128, 128, None) == 1    # Skv < 0
+        assert f(FAKE, FAKE, FAKE, None, FAKE, 4, 4, 2, 2, 64, 0.1, 128, 128, None) == 1     # o_parts
+        assert f(FAKE, FAKE, FAKE, FAKE + 8, FAKE, 4, 4, 2, 2, 64, 0.1, 128, 128, None) == 1
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE + 2, 4, 4, 2, 2, 64, 0.1, 128, 128, None) == 1  # lse_parts
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 2, 2, 96, 0.1, 128, 128, None) == 1     # d
+        assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 4, 2, 2, 64, 0.1, 120, 128, None) == 1     # ld_q
 
 
 def test_accumulate_rejects(lib):
