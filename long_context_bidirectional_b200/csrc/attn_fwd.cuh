@@ -8,18 +8,21 @@
 // 128-wide tiles with an online (running-max) softmax, the form ring
 // attention relies on (TensorRT 11.0 multi-device article, Ring Attention).
 //
-// Used for head dim 64, and for head dim 128 when a call has fewer than 96
+// Used for head dim 64, and for head dim 128 when a call has fewer than 48
 // key tiles (longer key ranges run on CTA pairs, attn_pair.cuh: this kernel's
 // pipeline fills and drains in fewer SM-cycles per row).  Both write their
 // results through attn_epilogue below, in the monolithic, partial or
 // accumulate (ring step) form.
-// One CTA owns two 128-row query tiles of one head.  Warp roles (18 warps):
+// One CTA owns two 128-row query tiles of one head and one key range: the
+// call's keys, or one of its P key chunks when a launch computes every
+// chunk's partial (CTA x = row block * P + chunk).  Warp roles (18 warps):
 //   warps 0-7   softmax for query tile 0, warps 8-15 for query tile 1.  Each
 //               row is shared by two threads (warps w and w+4 of a group, the
 //               same TMEM lane quarter), each owning 64 of the tile's 128
 //               score columns; the two exchange their row max through shared
 //               memory with a 64-thread named barrier.
-//   warp  16    TMA producer (Q once, then K_j, V_j through a smem ring)
+//   warp  16    TMA producer (Q once, then K_j, V_j through a smem ring;
+//               it also prefetches the next wave's Q tile into L2)
 //   warp  17    TMEM allocator and single-thread tcgen05.mma issuer
 // TMEM (512 columns x 128 lanes, fp32): S0 | S1 | O0 | O1.  The softmax
 // writes P (fp16, two per column) over the first half of its S block and the
