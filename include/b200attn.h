@@ -247,10 +247,10 @@ B2A_API int qkv_proj(const uint16_t* x, const uint16_t* w_qkv, uint16_t* qkv, in
 /*
  * qkv_proj_qknorm -- qkv_proj with the block's RMSNorm applied to q and k.
  *
- * The sample's block lists "Q/K/V projections, RMSNorm, scaled dot-product
- * attention, output projection" ("Multi-Device Attention Inference with
- * TensorRT", Generating the ONNX Models) without placement or epsilon; the
- * reading taken here normalises every head of q and of k after the
+ * The sample's block names an RMSNorm among its layers, after the Q/K/V
+ * projections and before the attention ("Multi-Device Attention Inference
+ * with TensorRT", Generating the ONNX Models), without placement or epsilon;
+ * the reading taken here normalises every head of q and of k after the
  * projection, in the GEMM's epilogue from the fp32 accumulator:
  *   q[i, h, :] <- q[i, h, :] / sqrt(mean_e q[i, h, e]^2 + eps) * g_q
  *   k[i, h, :] <- k[i, h, :] / sqrt(mean_e k[i, h, e]^2 + eps) * g_k

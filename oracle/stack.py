@@ -17,9 +17,9 @@ Readings where the pages are silent:
 * The block output is ``x + Z`` (a residual add).
 * RMSNorm, listed in the sample model without placement or epsilon, is not
   part of ``block``/``stack``.  ``qkv_qknorm`` gives the reading used when it
-  is asked for: the sample lists "Q/K/V projections, RMSNorm, scaled
-  dot-product attention, output projection" in that order, so the norm acts
-  on the projected q and k, per head, before attention (``qkv_qknorm``
+  is asked for: the sample names the norm after the Q/K/V projections and
+  ahead of the attention in its layer list, so the norm acts on the
+  projected q and k, per head, before attention (``qkv_qknorm``
   below; epsilon 1e-6 unless given, one weight vector of length d for q and
   one for k, shared by the heads).
 * Tensors are rounded to fp16 (round-to-nearest-even) exactly where the

@@ -1,17 +1,26 @@
 """CUDA stacked self-attention blocks against the FP64 oracle.
 
-Both sides start from the same seeded x and weights and round to fp16 at the
-same tensor boundaries (qkv, attention output, block output); nothing the
-GPU computes is fed to the oracle.  One-ulp rounding flips at those
-boundaries are expected (fp32 vs fp64 sums), so each compared tensor must
-meet rel_fro <= 1e-3 and, per element, |gpu - ref| <= max(4e-3, one fp16
-ulp of ref) when both sides start from identical inputs (block 1).  After
-block 1 each side feeds its own fp16 output forward: a flip persists along
-the residual stream, and a flipped q, k or v element moves the softmax
-weights of near-tied keys, so single elements of later blocks can drift
-apart by more than an ulp without any arithmetic error.  For blocks 2..6
-the bar is rel_fro <= 1e-3 on every tensor, plus a sanity bound of 2^-4 on
-any single element.
+Every block is checked from identical inputs: the GPU block i is given the
+same fp16 input the oracle's block i takes, so the comparison measures that
+block's arithmetic alone.  Nothing the GPU computes ever reaches the oracle.
+
+* S = 2048 (all rows): the oracle runs the whole 6-block chain; the GPU's
+  block i takes the oracle's fp16 output of block i-1 (block 1 takes x).
+* S = 32768 (256 sampled rows per block): the oracle's chain at this size is
+  out of reach of a test (each block's full attention is 1.8e13 FP64 flops),
+  so block 1 takes the seeded x and block i > 1 takes a fresh seeded
+  N(0, 1) fp16 input of the residual stream's shape; each block uses its own
+  weights.  The oracle evaluates the sampled rows (K and V from every row).
+
+Bars per block, on the fused qkv, the attention output and the block
+output: per element |gpu - ref| <= max(4e-3, one fp16 ulp of ref) (both sides
+round at the same tensor boundaries, so a one-ulp flip from fp32 vs fp64
+sums is allowed) and rel_fro <= 1e-3.
+
+The free-running chain (each side feeding its own output forward) is kept as
+a reported drift figure, held to rel_fro <= 1e-3 only: a one-ulp flip
+persists along the residual stream and moves the softmax weights of
+near-tied keys in later blocks.
 """
 import numpy as np
 import pytest
@@ -19,7 +28,7 @@ import torch
 
 import workloads as W
 from oracle import stack as OS
-from parity import REL_FRO, MAX_ABS, fp16_ulp, metrics
+from parity import REL_FRO, MAX_ABS, fp16_ulp, metrics, record
 
 pytestmark = pytest.mark.gpu
 
@@ -30,27 +39,61 @@ def b2a():
     return m
 
 
-def measure(gpu16, ref16, ulps=1):
+def measure(gpu16, ref16):
     """(worst error / per-element bound, max_abs, rel_fro)."""
     gpu = np.asarray(gpu16, dtype=np.float64)
     ref = np.asarray(ref16, dtype=np.float64)
     assert np.all(np.isfinite(gpu))
     err = np.abs(gpu - ref)
-    bound = np.maximum(MAX_ABS, ulps * fp16_ulp(ref))
+    bound = np.maximum(MAX_ABS, fp16_ulp(ref))
     ma, rf = metrics(gpu, ref)
     return float(np.max(err / bound)), ma, rf
 
 
-def check(gpu16, ref16, what, ulps=1):
-    worst, ma, rf = measure(gpu16, ref16, ulps)
+def check(gpu16, ref16, what):
+    worst, ma, rf = measure(gpu16, ref16)
+    record(what, "elem_bound", worst, 1.0)
+    record(what, "rel_fro", rf, REL_FRO)
     assert worst <= 1.0 and rf <= REL_FRO, f"{what}: worst {worst:.2f} of bound, max_abs={ma:.3e} rel_fro={rf:.3e}"
 
 
-def test_stack6_s2048_end_to_end(b2a):
+def gpu_block(b2a, x16, w_qkv, w_o, w):
+    """One block through the C ABI; returns (y, qkv, attention) on the host."""
+    S, h = x16.shape[0], w.hidden
+    qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device="cuda")
+    attn_ws = torch.empty((S, h), dtype=torch.float16, device="cuda")
+    y = b2a.attn_block_fwd(torch.from_numpy(x16).cuda(), w_qkv, w_o, w.H, w.d,
+                           qkv_ws=qkv_ws, attn_ws=attn_ws, scale=w.scale)
+    b2a.check_status()
+    return y.cpu().numpy(), qkv_ws.cpu().numpy(), attn_ws.cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def s2048_oracle_chain():
     w = W.STACK6_S2048
     x = W.stack_x(w)
     weights = [W.stack_weights(w, i) for i in range(w.blocks)]
-    ref = OS.stack(x, weights, w.H, w.d, w.scale)
+    return w, x, weights, OS.stack(x, weights, w.H, w.d, w.scale)
+
+
+def test_stack6_s2048_every_block_from_the_oracles_input(b2a, s2048_oracle_chain):
+    w, x, weights, ref = s2048_oracle_chain
+    inputs = [x] + [ref[i][0] for i in range(w.blocks - 1)]
+    fails = []
+    for i in range(w.blocks):
+        w_qkv, w_o = (torch.from_numpy(t).cuda() for t in weights[i])
+        y, qkv, a = gpu_block(b2a, inputs[i], w_qkv, w_o, w)
+        ry, rqkv, ra = ref[i]
+        for name, g, r in (("qkv", qkv, rqkv), ("attention", a, ra), ("output", y, ry)):
+            try:
+                check(g, r, f"s2048 block {i + 1} {name}")
+            except AssertionError as e:
+                fails.append(str(e))
+    assert not fails, "\n".join(fails)
+
+
+def test_stack6_s2048_free_running_drift(b2a, s2048_oracle_chain):
+    w, x, weights, ref = s2048_oracle_chain
     wd = [(torch.from_numpy(a).cuda(), torch.from_numpy(b).cuda()) for a, b in weights]
     kept = b2a.stack_forward(torch.from_numpy(x).cuda(), wd, w.H, w.d, scale=w.scale, keep=True)
     b2a.check_status()
@@ -58,26 +101,32 @@ def test_stack6_s2048_end_to_end(b2a):
     for i, ((y, qkv, a), (ry, rqkv, ra)) in enumerate(zip(kept, ref)):
         for name, g, r in (("qkv", qkv, rqkv), ("attention", a, ra), ("output", y, ry)):
             worst, ma, rf = measure(g.cpu().numpy(), r)
-            report.append(f"block {i + 1} {name}: {worst:.2f} of bound, max_abs={ma:.3e} rel_fro={rf:.3e}")
-            ok &= rf <= REL_FRO and (worst <= 1.0 if i == 0 else ma <= 2.0 ** -4)
+            record(f"s2048 free-running block {i + 1} {name}", "rel_fro", rf, REL_FRO)
+            report.append(f"block {i + 1} {name}: {worst:.2f} of the per-element bound, "
+                          f"max_abs={ma:.3e} rel_fro={rf:.3e}")
+            ok &= rf <= REL_FRO
     assert ok, "\n".join(report)
 
 
-def test_block1_s32768_sampled_rows(b2a):
+def stack32k_block_input(w, block):
+    """The input of block ``block`` at S = 32768 (see the module docstring)."""
+    if block == 0:
+        return W.stack_x(w)
+    return W.stack_x(W.StackWorkload(w.name, w.S, w.H, w.d, w.blocks, w.w_sigma, seed=300 + block))
+
+
+@pytest.mark.parametrize("block", range(6))
+def test_stack6_s32768_block_sampled_rows(b2a, block):
     w = W.STACK6
-    x = W.stack_x(w)
-    w_qkv, w_o = W.stack_weights(w, 0)
-    xd = torch.from_numpy(x).cuda()
-    qkv_ws = torch.empty((w.S, 3 * w.hidden), dtype=torch.float16, device="cuda")
-    attn_ws = torch.empty((w.S, w.hidden), dtype=torch.float16, device="cuda")
-    y = b2a.attn_block_fwd(xd, torch.from_numpy(w_qkv).cuda(), torch.from_numpy(w_o).cuda(), w.H, w.d,
-                           qkv_ws=qkv_ws, attn_ws=attn_ws, scale=w.scale)
-    b2a.check_status()
-    rows = W.sample_rows(w.S, 1, 0, seed=7)
+    assert block < w.blocks
+    x = stack32k_block_input(w, block)
+    w_qkv, w_o = W.stack_weights(w, block)
+    y, qkv, a = gpu_block(b2a, x, torch.from_numpy(w_qkv).cuda(), torch.from_numpy(w_o).cuda(), w)
+    rows = W.sample_rows(w.S, 1, block, seed=7)
     ry, rqkv, ra = OS.block_rows(x, w_qkv, w_o, w.H, w.d, w.scale, rows)
-    check(qkv_ws.cpu().numpy()[rows], rqkv, "block 1 qkv (sampled rows)")
-    check(attn_ws.cpu().numpy()[rows], ra, "block 1 attention (sampled rows)")
-    check(y.cpu().numpy()[rows], ry, "block 1 output (sampled rows)")
+    check(qkv[rows], rqkv, f"32k block {block + 1} qkv (sampled rows)")
+    check(a[rows], ra, f"32k block {block + 1} attention (sampled rows)")
+    check(y[rows], ry, f"32k block {block + 1} output (sampled rows)")
 
 
 def test_block_with_qk_rmsnorm(b2a):
