@@ -50,6 +50,8 @@ def parse():
                     help="override the workload's number of KV chunks P")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration side measurements")
     ap.add_argument("--attn-kernel", default="auto", choices=["auto", "single", "pair"],
                     help="head-dim-128 attention kernel (default: chosen by key count)")
     return ap.parse_args()
@@ -242,6 +244,57 @@ def cpu_baseline(w, budget_s: float = 10.0):
 
 # --------------------------------------------------------------- our arm --
 
+def measure_attn_config(b2a, w, dev, stream, world, pk, n=5):
+    """One attention workload, CUDA-event timed: monolithic attn_fwd and, for
+    workloads with P > 1 key chunks, the partials launch and the merge."""
+    import torch
+    q, k, v = W.workload_qkv(w)
+    qd, kd, vd = (torch.from_numpy(x).to(dev) for x in (q, k, v))
+    S, H, d = w.S, w.H, w.d
+    out = torch.empty((S, H, d), dtype=torch.float16, device=dev)
+    lse = torch.empty((H, S), dtype=torch.float32, device=dev)
+
+    def timed(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        b2a.check_status(stream)
+        return reduce_max(a.elapsed_time(b) / reps, world)
+
+    mono_ms = timed(lambda: b2a.attn_fwd(qd, kd, vd, out=out, lse=lse, scale=w.scale, stream=stream), n)
+    tfl = w.flops / (mono_ms * 1e-3) / 1e12
+    res = {"S": S, "H": H, "d": d, "q_sigma": w.q_sigma, "attn_kernel": attn_kernel_name(b2a, d, S),
+           "attn_fwd_ms": mono_ms, "attn_fwd_tflops": tfl, "attn_fwd_frac": tfl / pk["tc_burst"]}
+    if w.P > 1:
+        P = w.P
+        o_parts = torch.empty((P, S, H, d), dtype=torch.float32, device=dev)
+        lse_parts = torch.empty((P, H, S), dtype=torch.float32, device=dev)
+        part_ms = timed(lambda: b2a.attn_fwd_partials(qd, kd, vd, P, o_parts, lse_parts, scale=w.scale,
+                                                      stream=stream), n)
+        out_c = torch.empty_like(out)
+        lse_c = torch.empty_like(lse)
+        merge_ms = timed(lambda: b2a.attn_merge(o_parts, lse_parts, out=out_c, lse_out=lse_c, stream=stream),
+                         4 * n)
+        merge_bytes = P * S * H * d * 4 + P * H * S * 4 + S * H * d * 2 + H * S * 4
+        ptf = w.flops / (part_ms * 1e-3) / 1e12
+        gbs = merge_bytes / (merge_ms * 1e-3) / 1e9
+        res.update({"P": P, "partials_ms": part_ms, "partials_tflops": ptf, "partials_frac": ptf / pk["tc_burst"],
+                    "partials_kernel": attn_kernel_name(b2a, d, (S + P - 1) // P, 1),
+                    "merge_ms": merge_ms, "merge_gbs": gbs, "merge_hbm_frac": gbs / pk["hbm_gbs"],
+                    "step_ms": mono_ms + part_ms + merge_ms,
+                    "step_tflops": 2 * w.flops / ((mono_ms + part_ms + merge_ms) * 1e-3) / 1e12})
+    res["peaks"] = "tensor-bound kernels against the burst bf16 figure, the merge against the copy bandwidth"
+    return res
+
+
+
 def run_ours(args, rank, world, local):
     import torch
     import long_context_bidirectional_b200 as b2a
@@ -424,9 +477,24 @@ def run_ours(args, rank, world, local):
     p16_ms = time_calls(part16_pass, n=3)
     m16_ms = time_calls(lambda: b2a.attn_merge_f16(o16_parts, lse_parts, out=out_c, lse_out=lse_c,
                                                    stream=stream))
-    del o16_parts
     merge16_bytes = P * S * H * d * 2 + P * H * S * 4 + S * H * d * 2 + H * S * 4
     merge16_gbs = merge16_bytes / (m16_ms * 1e-3) / 1e9
+
+    # The other configurations of the pages' validation tables, each timed
+    # with CUDA events on its own inputs (not part of ``value``): S=8192 at
+    # hidden 4096 (monolithic + 2 key chunks + merge), S=65536 at hidden
+    # 4096, S=8192 at hidden 8192 (64 heads), and the 6-block stack at
+    # S=32768 with its attention and projection GEMMs reported separately.
+    configs = {}
+    if not args.no_configs:
+        del o16_parts
+        for cw in (W.SEQ8K, W.SEQ64K, W.SEQ8K_H64):
+            configs[cw.name] = measure_attn_config(b2a, cw, dev, stream, world, pk)
+            torch.cuda.empty_cache()
+        configs[W.STACK6.name] = measure_stack(b2a, W.STACK6, dev, stream, steps=3, warmup=2, world=world)
+        torch.cuda.empty_cache()
+    else:
+        del o16_parts
 
     # end to end from pinned host memory through the C-ABI host entry point
     e2e = None
@@ -516,6 +584,7 @@ def run_ours(args, rank, world, local):
                     "merge_f16_ms": m16_ms, "merge_f16_gbs": merge16_gbs,
                     "merge_f16_hbm_frac": merge16_gbs / pk["hbm_gbs"], "merge_f16_bytes": merge16_bytes,
                     "fp16_split_reduction": "attn_fwd_partials_f16 + attn_merge_f16 (not in value)"},
+        "configs": configs,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * (part_launches + 2),
@@ -527,24 +596,18 @@ def run_ours(args, rank, world, local):
 
 # ------------------------------------------------------- stack workload --
 
-def run_stack(args, rank, world, local):
-    """Six stacked self-attention blocks (fused QKV GEMM, attention on strided
-    views, output GEMM + residual) on x [S, H*d]; value counts attention plus
-    both projections."""
+def measure_stack(b2a, w, dev, stream, steps, warmup, world, sample_clocks=False):
+    """Time ``w.blocks`` stacked blocks (fused QKV GEMM, attention on strided
+    views of its output, output GEMM + residual) on x [S, H*d]: the whole
+    step from CUDA events around it, and each kernel's share from events
+    around every launch.  Returns the figures as a dict."""
     import torch
-    import long_context_bidirectional_b200 as b2a
-
-    w = W.STACK_WORKLOADS[args.workload]
-    b2a.set_attn_kernel(ATTN_KERNEL_CHOICE[args.attn_kernel])
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
     S, H, d, h = w.S, w.H, w.d, w.hidden
     x0 = torch.from_numpy(W.stack_x(w)).to(dev)
     weights = [tuple(torch.from_numpy(t).to(dev) for t in W.stack_weights(w, i)) for i in range(w.blocks)]
     x = torch.empty_like(x0)
     qkv_ws = torch.empty((S, 3 * h), dtype=torch.float16, device=dev)
     attn_ws = torch.empty((S, h), dtype=torch.float16, device=dev)
-    stream = torch.cuda.current_stream(dev)
     ev = []
 
     def step(record):
@@ -566,34 +629,51 @@ def run_stack(args, rank, world, local):
                 e[3].record(stream)
                 ev.append(e)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step(False)
     b2a.check_status(stream)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(bus_id_of(local)) as clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(args.steps):
-            step(True)
-        t1.record(stream)
-        torch.cuda.synchronize()
+    clk = ClockSampler(bus_id_of(dev.index)) if sample_clocks else None
+    if clk:
+        clk.__enter__()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__(None, None, None)
     barrier(world)
     b2a.check_status(stream)
-    ms = reduce_max(t0.elapsed_time(t1) / args.steps, world)
+    ms = reduce_max(t0.elapsed_time(t1) / steps, world)
     n = len(ev)
-    qkv_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / n
-    att_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / n
-    out_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / n
+    qkv_ms = reduce_max(sum(e[0].elapsed_time(e[1]) for e in ev) / n, world)
+    att_ms = reduce_max(sum(e[1].elapsed_time(e[2]) for e in ev) / n, world)
+    out_ms = reduce_max(sum(e[2].elapsed_time(e[3]) for e in ev) / n, world)
     f_att = 4.0 * S * S * d * H
     f_qkv = 2.0 * S * 3 * h * h
     f_out = 2.0 * S * h * h
     step_flops = w.blocks * (f_att + f_qkv + f_out)
     pk = peaks()
 
+    def tf(f, t):
+        return f / (t * 1e-3) / 1e12
+
+    res = {"workload": w.name, "S": S, "H": H, "d": d, "blocks": w.blocks, "ms_per_step": ms,
+           "step_flops": step_flops, "tflops": job_throughput(world, step_flops, ms) / 1e12,
+           "frac": tf(step_flops, ms) / pk["tc_burst"],
+           "qkv_proj_ms": qkv_ms, "qkv_proj_tflops": tf(f_qkv, qkv_ms), "qkv_proj_frac": tf(f_qkv, qkv_ms) / pk["tc_burst"],
+           "attn_fwd_ms": att_ms, "attn_fwd_tflops": tf(f_att, att_ms), "attn_fwd_frac": tf(f_att, att_ms) / pk["tc_burst"],
+           "attn_kernel": attn_kernel_name(b2a, d, S),
+           "out_proj_ms": out_ms, "out_proj_tflops": tf(f_out, out_ms), "out_proj_frac": tf(f_out, out_ms) / pk["tc_burst"],
+           "peak": pk["tc_burst"], "peak_source": pk["source"] + "; burst figure"}
+    if clk:
+        res["clocks"] = clk.summary()
     # The projection with the q/k RMSNorm epilogue (the norm reading of the
-    # sample block), timed on its own; not part of ``value``.
+    # sample block), timed on its own; not part of the step.
     g_ones = torch.ones(d, dtype=torch.float16, device=dev)
     for _ in range(2):
         b2a.qkv_proj_qknorm(x0, weights[0][0], g_ones, g_ones, H, d, 1e-6, out=qkv_ws, stream=stream)
@@ -607,26 +687,41 @@ def run_stack(args, rank, world, local):
     torch.cuda.synchronize()
     b2a.check_status(stream)
     qkn_ms = reduce_max(na.elapsed_time(nb_) / 5, world)
+    res["qkv_proj_qknorm_ms"] = qkn_ms
+    res["qkv_proj_qknorm_tflops"] = tf(f_qkv, qkn_ms)
+    del x0, weights, x, qkv_ws, attn_ws
+    return res
+
+
+def run_stack(args, rank, world, local):
+    """Six stacked self-attention blocks (fused QKV GEMM, attention on strided
+    views, output GEMM + residual) on x [S, H*d]; value counts attention plus
+    both projections."""
+    import torch
+    import long_context_bidirectional_b200 as b2a
+
+    w = W.STACK_WORKLOADS[args.workload]
+    b2a.set_attn_kernel(ATTN_KERNEL_CHOICE[args.attn_kernel])
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    r = measure_stack(b2a, w, dev, stream, args.steps, args.warmup, world, sample_clocks=True)
+    pk = peaks()
     line = {
-        "metric": METRIC, "value": job_throughput(world, step_flops, ms) / 1e12, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "metric": METRIC, "value": r["tflops"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": {"workload": w.name, "S": S, "H": H, "d": d, "blocks": w.blocks, "batch": 1,
+        "config": {"workload": w.name, "S": w.S, "H": w.H, "d": w.d, "blocks": w.blocks, "batch": 1,
                    "step": "per block: qkv_proj, attn_fwd on strided views, out_proj + residual",
-                   "step_flops": step_flops, "l2": "inputs larger than L2 (weights 128 MiB per block)",
+                   "step_flops": r["step_flops"], "l2": "inputs larger than L2 (weights 128 MiB per block)",
                    "parallelism": f"replicas x{world}"},
-        "kernels": {"qkv_proj_ms": qkv_ms, "qkv_proj_tflops": f_qkv / (qkv_ms * 1e-3) / 1e12,
-                    "attn_fwd_ms": att_ms, "attn_fwd_tflops": f_att / (att_ms * 1e-3) / 1e12,
-                    "out_proj_ms": out_ms, "out_proj_tflops": f_out / (out_ms * 1e-3) / 1e12,
-                    "qkv_proj_qknorm_ms": qkn_ms, "qkv_proj_qknorm_tflops": f_qkv / (qkn_ms * 1e-3) / 1e12,
-                    "qkv_proj_qknorm": "qkv projection with the q/k RMSNorm epilogue (not in value)"},
-        "roofline": {"bound": "tensor", "kernel": attn_kernel_name(b2a, d, S),
-                     "achieved": f_att / (att_ms * 1e-3) / 1e12, "peak": pk["tc_burst"], "unit": "TFLOP/s",
-                     "frac": f_att / (att_ms * 1e-3) / 1e12 / pk["tc_burst"], "peak_source": pk["source"],
-                     "traffic": None, "algorithmic": "4*S^2*d*H flops per launch"},
+        "kernels": {k: v for k, v in r.items() if k.startswith(("qkv_proj", "attn_fwd", "out_proj"))},
+        "roofline": {"bound": "tensor", "kernel": r["attn_kernel"], "achieved": r["attn_fwd_tflops"],
+                     "peak": pk["tc_burst"], "unit": "TFLOP/s", "frac": r["attn_fwd_frac"],
+                     "peak_source": pk["source"], "traffic": None, "algorithmic": "4*S^2*d*H flops per launch"},
         "cpu_baseline": None, "e2e": None,
         "gpu_launches": args.steps * w.blocks * 3,
-        "clocks": clk.summary(),
+        "clocks": r.get("clocks"),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
