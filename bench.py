@@ -187,6 +187,14 @@ def attn_kernel_name(b2a, d: int, Skv: int, mode: int = 0) -> str:
     return f"attn_fwd_kernel<{d}, {mode}, 0>"
 
 
+def merge_kernel_name(d: int, P: int, partial_type: str) -> str:
+    """The merge kernel the library launches: the pipelined persistent form
+    up to 16 chunks, else the one-group-per-block form."""
+    if P <= 16:
+        return f"attn_merge_pipe_kernel<{d}, {partial_type}>"
+    return f"attn_merge_kernel<{d}, {partial_type}>"
+
+
 def committed_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if it matches the source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -243,6 +251,32 @@ def cpu_baseline(w, budget_s: float = 10.0):
 
 
 # --------------------------------------------------------------- our arm --
+
+def measure_batched(b2a, S, B, H, d, dev, stream, world, pk, n=5):
+    """attn_fwd_batched on the (S, B, hidden) layout, one launch over every
+    (row block, head, batch); inputs seeded like the attention workloads."""
+    import torch
+    q, k, v = W.qkv(S, B * H, d, seed=0)
+    qd, kd, vd = (torch.from_numpy(x).to(dev).view(S, B, H, d) for x in (q, k, v))
+    out = torch.empty_like(qd)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    fn = lambda: b2a.attn_fwd_batched(qd, kd, vd, out=out, lse=lse, scale=1 / math.sqrt(d), stream=stream)
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    b2a.check_status(stream)
+    ms = reduce_max(a.elapsed_time(b) / n, world)
+    tfl = 4.0 * S * S * d * H * B / (ms * 1e-3) / 1e12
+    return {"S": S, "B": B, "H": H, "d": d, "attn_fwd_batched_ms": ms, "attn_fwd_batched_tflops": tfl,
+            "attn_fwd_batched_frac": tfl / pk["tc_burst"], "launches": 1}
+
 
 def measure_attn_config(b2a, w, dev, stream, world, pk, n=5):
     """One attention workload, CUDA-event timed: monolithic attn_fwd and, for
@@ -386,7 +420,7 @@ def run_ours(args, rank, world, local):
          "unit": "TFLOP/s", "peak": pk["tc_burst"],
          "algorithmic": ("4*S^2*d*H flops per launch (all chunks)" if one_launch
                          else "4*S*(S/P)*d*H flops per launch (one chunk)")},
-        {"bound": "hbm", "kernel": f"attn_merge_kernel<{d}, float>", "role": "attn_merge",
+        {"bound": "hbm", "kernel": merge_kernel_name(d, P, "float"), "role": "attn_merge",
          "launches_per_step": 1, "ms_per_launch": merge_ms, "achieved": merge_gbs, "unit": "GB/s",
          "peak": pk["hbm_gbs"],
          "algorithmic": "P*S*H*d*4 + P*H*S*4 + S*H*d*2 + H*S*4 bytes per launch (o_parts, lse_parts, out, lse)"},
@@ -492,6 +526,8 @@ def run_ours(args, rank, world, local):
             configs[cw.name] = measure_attn_config(b2a, cw, dev, stream, world, pk)
             torch.cuda.empty_cache()
         configs[W.STACK6.name] = measure_stack(b2a, W.STACK6, dev, stream, steps=3, warmup=2, world=world)
+        torch.cuda.empty_cache()
+        configs["batched_s8192_b4_h32_d128"] = measure_batched(b2a, 8192, 4, 32, 128, dev, stream, world, pk)
         torch.cuda.empty_cache()
     else:
         del o16_parts

@@ -46,7 +46,8 @@ typedef enum {
   B2A_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, stride or scale */
   B2A_ERR_UNSUPPORTED = 2, /* not an sm_100 device, or a size beyond an implementation limit */
   B2A_ERR_CUDA = 3,        /* a CUDA runtime call failed; see b2a_last_cuda_error() */
-  B2A_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (reported by b2a_check_status) */
+  B2A_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (reported by b2a_check_status) */
+  B2A_ERR_DEVICE_CHECK = 5 /* debug build: a device-side bounds check failed (reported by b2a_check_status) */
 } b2a_status;
 
 /*
@@ -77,11 +78,14 @@ B2A_API int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, ui
  * activation layout ("Multi-Device Attention Inference with TensorRT",
  * Generating the ONNX Models: input/output (sequence_length, batch_size,
  * 4096)).  Batch b is the strided view that starts at column b*H*d with row
- * stride B*H*d; the call runs attn_fwd on each batch in turn on `stream`.
+ * stride B*H*d.  Heads of different batches are independent, so [S, B, H, d]
+ * is taken as [S, B*H, d] (batch b's head h = head b*H + h, lse [B*H, S]) and
+ * one launch covers every (row block, head, batch).  Results equal attn_fwd
+ * on each batch's view, bit for bit.
  *
  * q, k, v, out  device fp16 [S, B, H, d] contiguous.
  * lse           device fp32 [B, H, S], or NULL.
- * B >= 1 and B*H*d <= 2^31 - 1; other requirements as attn_fwd.
+ * B >= 1, B*H <= 65535 and B*H*d <= 2^31 - 1; other requirements as attn_fwd.
  */
 B2A_API int attn_fwd_batched(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                              float* lse, int S, int B, int H, int d, float scale, void* stream);
@@ -379,9 +383,11 @@ B2A_API uint64_t attn_fwd_host_workspace_bytes(int S, int H, int d, int P);
 
 /*
  * b2a_check_status -- synchronise `stream`, then read and clear the device
- * status word that kernels set when a bounded wait runs out.  Returns
- * B2A_OK, B2A_ERR_TIMEOUT, or B2A_ERR_CUDA if the synchronisation failed.
- * Blocks the calling host thread.
+ * status word that kernels set when a bounded wait runs out or, in the
+ * debug build, when a bounds check fails.  Returns B2A_OK,
+ * B2A_ERR_DEVICE_CHECK (a bounds check failed; waits that then gave up are
+ * its consequence), B2A_ERR_TIMEOUT, or B2A_ERR_CUDA if the synchronisation
+ * failed.  Blocks the calling host thread.
  */
 B2A_API int b2a_check_status(void* stream);
 
@@ -429,6 +435,22 @@ B2A_API int b2a_get_attn_kernel(void);
 B2A_API int b2a_attn_kernel_for(int d, int Skv);
 
 /* Library ABI version (major*100 + minor). */
+/*
+ * b2a_debug_build -- 1 if this library is the debug build
+ * (libb200attn_debug.so, compiled with -DB2A_DEBUG), else 0.  The pages have
+ * no counterpart: the debug build is this library's stand-in for a memory
+ * checker.  Before every tiled TMA copy it checks the box's start against
+ * the tensor map's extents (the innermost coordinate also for 16-byte
+ * alignment) and the destination against the CTA's shared memory; before
+ * every tcgen05.ld / tcgen05.st / tcgen05.mma it checks the TMEM lane field
+ * and columns against the 512-column allocation.  A failed check skips the
+ * access, ORs a bit into the device status word (the kernel's waits then give
+ * up at once and it returns) and b2a_check_status() returns
+ * B2A_ERR_DEVICE_CHECK.  Same entry points and results as the release build,
+ * slower.
+ */
+B2A_API int b2a_debug_build(void);
+
 B2A_API int b2a_version(void);
 
 #ifdef __cplusplus

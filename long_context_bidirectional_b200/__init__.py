@@ -19,7 +19,11 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libb200attn.so")
+# ATTN_DEBUG=1 selects the debug build (every TMA box and TMEM access
+# bounds-checked on the device before it is issued; same entry points).
+_DEBUG = os.environ.get("ATTN_DEBUG", "0") not in ("", "0")
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib",
+                         "libb200attn_debug.so" if _DEBUG else "libb200attn.so")
 
 __all__ = [
     "B2AError", "lib", "attn_fwd", "attn_fwd_batched", "attn_fwd_gathered_kv", "attn_fwd_partial", "attn_fwd_accumulate",
@@ -30,7 +34,7 @@ __all__ = [
     "chunk_bounds", "library_path",
 ]
 
-B2A_OK, B2A_ERR_INVALID_ARG, B2A_ERR_UNSUPPORTED, B2A_ERR_CUDA, B2A_ERR_TIMEOUT = range(5)
+B2A_OK, B2A_ERR_INVALID_ARG, B2A_ERR_UNSUPPORTED, B2A_ERR_CUDA, B2A_ERR_TIMEOUT, B2A_ERR_DEVICE_CHECK = range(6)
 ATTN_KERNEL_AUTO, ATTN_KERNEL_SINGLE, ATTN_KERNEL_PAIR = range(3)
 
 _u16p = ctypes.c_void_p
@@ -65,6 +69,7 @@ _SIGS = {
     "b2a_status_string": (ctypes.c_char_p, [_i]),
     "b2a_last_cuda_error": (_i, []),
     "b2a_version": (_i, []),
+    "b2a_debug_build": (_i, []),
 }
 
 

@@ -20,6 +20,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIBDIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIBDIR, "libb200attn.so")
+# The debug build (-DB2A_DEBUG): every TMA box and TMEM access bounds-checked
+# on the device before issue; selected in the binding by ATTN_DEBUG=1.
+DEBUG_LIB = os.path.join(LIBDIR, "libb200attn_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -33,21 +36,26 @@ def nvcc() -> str:
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                  + glob.glob(os.path.join(CSRC, "*.h"))
                   + [os.path.join(INCLUDE, "b200attn.h")])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
+    """Compile the release library, or with ``debug`` the bounds-checked one."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
     os.makedirs(LIBDIR, exist_ok=True)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
+    if debug:
+        extra_flags = ("-DB2A_DEBUG", *extra_flags)
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-shared", "-cudart", "static", f"-I{INCLUDE}", f"-I{CSRC}",
@@ -61,10 +69,21 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose:
         print(res.stderr, file=sys.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
+
+
+def build_all(force: bool = False) -> None:
+    """Both libraries, compiled concurrently."""
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(2) as ex:
+        for f in [ex.submit(build, force, False, (), dbg) for dbg in (False, True)]:
+            f.result()
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
-    print(build(force=force, verbose="-v" in sys.argv))
+    if "--debug" in sys.argv:
+        print(build(force=force, verbose="-v" in sys.argv, debug=True))
+    else:
+        print(build(force=force, verbose="-v" in sys.argv))

@@ -422,13 +422,15 @@ __global__ void __launch_bounds__(576, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      // end of the query rows this grid covers (debug-build bounds)
+      const int q_rows_end = (p.Sq + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA * C::ROWS_PER_CTA;
       mbar_arrive_expect_tx(bar(C::B_Q), C::QT * C::Q_BYTES);
 #pragma unroll
       for (int qt = 0; qt < C::QT; ++qt)
 #pragma unroll
         for (int sb = 0; sb < C::SUB; ++sb)
-          tma_load_3d(sQ + qt * C::Q_BYTES + sb * C::SUB_BYTES, &tm_q, bar(C::B_Q), sb * 64, head,
-                      q0 + qt * C::BM);
+          tma_load_3d_chk(sQ + qt * C::Q_BYTES + sb * C::SUB_BYTES, C::SUB_BYTES, raw_u32, &tm_q, bar(C::B_Q),
+                          sb * 64, head, q0 + qt * C::BM, D, p.H, q_rows_end);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
@@ -445,8 +447,8 @@ __global__ void __launch_bounds__(576, 1)
           const CUtensorMap* m = kind ? &tm_v : &tm_k;
 #pragma unroll
           for (int sb = 0; sb < C::SUB; ++sb)
-            tma_load_3d(sKV + st * C::KV_BYTES + sb * C::SUB_BYTES, m, bar(C::B_KVF + st), sb * 64,
-                        head, key0 + j * C::BN);
+            tma_load_3d_chk(sKV + st * C::KV_BYTES + sb * C::SUB_BYTES, C::SUB_BYTES, raw_u32, m,
+                            bar(C::B_KVF + st), sb * 64, head, key0 + j * C::BN, D, p.H, key0 + klen);
           ++issued;
         }
         if (j == 0 && p.wave > 0) {

@@ -159,10 +159,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      // ends of the query and key rows this launch covers (debug-build bounds)
+      const int q_rows_end = (p.Sq + C::ROWS_PER_PAIR - 1) / C::ROWS_PER_PAIR * C::ROWS_PER_PAIR;
+      const int kv_rows_end = nkv * C::BN;
       if (leader) mbar_arrive_expect_tx(bar(C::B_Q), 2 * C::Q_BYTES);
       const uint32_t lq = map_to_rank(bar(C::B_Q), 0);
 #pragma unroll
-      for (int sb = 0; sb < 2; ++sb) tma_load_3d_pair(sQ + sb * C::QSUB, &tm_q, lq, sb * 64, head, q0);
+      for (int sb = 0; sb < 2; ++sb)
+        tma_load_3d_pair_chk(sQ + sb * C::QSUB, C::QSUB, raw_u32, &tm_q, lq, sb * 64, head, q0, D, p.H, q_rows_end);
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
@@ -177,8 +181,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         const uint32_t dst = sKV + st * C::STAGE_BYTES;
 #pragma unroll
         for (int sb = 0; sb < 2; ++sb)
-          tma_load_3d_pair(dst + sb * C::KSUB, &tm_k, lf, sb * 64, head, j * C::BN + static_cast<int>(rank) * 64);
-        tma_load_3d_pair(dst + C::KH_BYTES, &tm_v, lf, static_cast<int>(rank) * 64, head, j * C::BN);
+          tma_load_3d_pair_chk(dst + sb * C::KSUB, C::KSUB, raw_u32, &tm_k, lf, sb * 64, head,
+                               j * C::BN + static_cast<int>(rank) * 64, D, p.H, kv_rows_end);
+        tma_load_3d_pair_chk(dst + C::KH_BYTES, C::VH_BYTES, raw_u32, &tm_v, lf, static_cast<int>(rank) * 64, head,
+                             j * C::BN, D, p.H, kv_rows_end);
         ++issued;
       }
       // The leader's barriers count both CTAs' bytes; after a failed wait

@@ -21,10 +21,6 @@
 
 namespace {
 
-// Set by kernels when a bounded wait runs out; read and cleared by
-// b2a_check_status().  One word per device (static device memory).
-__device__ unsigned int g_status_word;
-
 thread_local int t_last_cuda_error = 0;
 
 int cuda_fail(cudaError_t e) {
@@ -65,7 +61,7 @@ int current_device(const DeviceInfo** info) {
     di.sm_count = sms;
     if (di.supported) {
       void* p = nullptr;
-      if ((e = cudaGetSymbolAddress(&p, g_status_word)) != cudaSuccess) return cuda_fail(e);
+      if ((e = cudaGetSymbolAddress(&p, b2a::g_status_word)) != cudaSuccess) return cuda_fail(e);
       di.status = static_cast<unsigned int*>(p);
     }
     di.probed = true;
@@ -422,6 +418,18 @@ int launch_merge(const T* o_parts, const float* lse_parts, int P, uint16_t* out,
   const DeviceInfo* di = nullptr;
   int st = current_device(&di);
   if (st != B2A_OK) return st;
+#ifndef B2A_MERGE_PIPE
+#define B2A_MERGE_PIPE 1
+#endif
+  if (B2A_MERGE_PIPE && P <= b2a::kMergePipeMaxP) {
+    // persistent, two blocks per SM, weights of the next pair group computed
+    // while the current one streams
+    auto pk = d == 128 ? b2a::attn_merge_pipe_kernel<128, T> : b2a::attn_merge_pipe_kernel<64, T>;
+    const long long grid = blocks < 2LL * di->sm_count ? blocks : 2LL * di->sm_count;
+    pk<<<static_cast<unsigned>(grid), b2a::kMergePairs, 0, stream>>>(o_parts, lse_parts, P, S, H, out, lse_out);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? B2A_OK : cuda_fail(e);
+  }
   const int smem = P * b2a::kMergePairs * static_cast<int>(sizeof(float));
   auto kern = d == 128 ? b2a::attn_merge_kernel<128, T> : b2a::attn_merge_kernel<64, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -609,19 +617,15 @@ int attn_fwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* 
 
 int attn_fwd_batched(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse, int S,
                      int B, int H, int d, float scale, void* stream) {
+  // [S, B, H, d] is [S, B*H, d] with row stride B*H*d: batch b's head h is
+  // head b*H + h, and lse [B, H, S] is [B*H, S].  One launch covers every
+  // (row block, head, batch).
   if (B < 1 || H < 1 || S < 1) return B2A_ERR_INVALID_ARG;
-  const long long row = static_cast<long long>(B) * H * d;
-  if (row > INT_MAX) return B2A_ERR_UNSUPPORTED;
-  const int ld = static_cast<int>(row);
-  const size_t hd = static_cast<size_t>(H) * d;
-  for (int b = 0; b < B; ++b) {
-    const size_t off = static_cast<size_t>(b) * hd;
-    float* lse_b = lse ? lse + static_cast<size_t>(b) * H * S : nullptr;
-    const int st = attn_fwd_impl(q + off, k + off, v + off, out + off, lse_b, S, S, H, d, scale, ld, ld, ld, ld,
-                                 static_cast<cudaStream_t>(stream));
-    if (st != B2A_OK) return st;
-  }
-  return B2A_OK;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh * d > INT_MAX) return B2A_ERR_UNSUPPORTED;
+  const int ld = static_cast<int>(bh * d);
+  return attn_fwd_impl(q, k, v, out, lse, S, S, static_cast<int>(bh), d, scale, ld, ld, ld, ld,
+                       static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_gathered_kv(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
@@ -867,7 +871,8 @@ int b2a_check_status(void* stream) {
   const unsigned int zero = 0;
   if ((e = cudaMemcpy(di->status, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(e);
-  return B2A_ERR_TIMEOUT;
+  // a failed bounds check (debug builds) is the cause of any wait that then gave up
+  return (v & b2a::kDevErrBounds) ? B2A_ERR_DEVICE_CHECK : B2A_ERR_TIMEOUT;
 }
 
 const char* b2a_status_string(int status) {
@@ -877,13 +882,16 @@ const char* b2a_status_string(int status) {
     case B2A_ERR_UNSUPPORTED: return "unsupported device or size";
     case B2A_ERR_CUDA: return "CUDA runtime error";
     case B2A_ERR_TIMEOUT: return "device-side wait timed out";
+    case B2A_ERR_DEVICE_CHECK: return "device-side bounds check failed (debug build)";
     default: return "unknown status";
   }
 }
 
 int b2a_last_cuda_error(void) { return t_last_cuda_error; }
 
-int b2a_version(void) { return 103; }
+int b2a_version(void) { return 104; }
+
+int b2a_debug_build(void) { return b2a::kDebugBuild ? 1 : 0; }
 
 #ifdef B2A_TRACE
 // Trace builds only: choose the traced CTA, then read the event table

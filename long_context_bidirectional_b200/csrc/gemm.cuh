@@ -242,6 +242,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     if (lane == 0) {
       prefetch_tmap(&tm_a);
       prefetch_tmap(&tm_b);
+      // ends of the K columns and of the A / W rows the tiles cover
+      // (debug-build bounds)
+      const int k_end = nk * C::BK;
+      const int m_end = p.tiles_m * C::PAIR_M, n_end = p.tiles_n * C::BN;
       int it = 0;
       bool ok = true;
       for (int tile = cluster; tile < p.num_tiles && ok; tile += nclusters) {
@@ -261,8 +265,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const uint32_t sa = sBase + st * C::STAGE_BYTES;
 #pragma unroll
           for (int sb = 0; sb < C::BK / C::KSUB; ++sb) {
-            tma_load_2d_pair(sa + sb * C::A_SUB, &tm_a, lf, kb * C::BK + sb * C::KSUB, arow);
-            tma_load_2d_pair(sa + C::A_BYTES + sb * C::B_SUB, &tm_b, lf, kb * C::BK + sb * C::KSUB, brow);
+            tma_load_2d_pair_chk(sa + sb * C::A_SUB, C::A_SUB, raw_u32, &tm_a, lf, kb * C::BK + sb * C::KSUB, arow,
+                                 k_end, m_end);
+            tma_load_2d_pair_chk(sa + C::A_BYTES + sb * C::B_SUB, C::B_SUB, raw_u32, &tm_b, lf,
+                                 kb * C::BK + sb * C::KSUB, brow, k_end, n_end);
           }
         }
       }

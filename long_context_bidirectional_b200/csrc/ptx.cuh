@@ -9,12 +9,47 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
+#include "debug_checks.h"
+
 namespace b2a {
 
 // Status bits OR-ed into the device status word by kernels.
 enum : uint32_t {
   kDevErrTimeout = 1u,      // a bounded mbarrier wait ran out
+  kDevErrBounds = 2u,       // a debug-build bounds check failed (the access was skipped)
 };
+
+// The library's device status word (one per device, static device memory):
+// set by kernels, read and cleared by b2a_check_status().
+__device__ unsigned int g_status_word;
+
+#ifdef B2A_DEBUG
+constexpr bool kDebugBuild = true;
+#else
+constexpr bool kDebugBuild = false;
+#endif
+
+// Debug builds: a failed check sets kDevErrBounds and returns false, and the
+// caller skips the access.  Release builds: always true, the check compiles
+// away.
+__device__ __forceinline__ bool dbg_check(bool ok) {
+  if constexpr (kDebugBuild) {
+    if (!ok) {
+      atomicOr(&g_status_word, kDevErrBounds);
+      return false;
+    }
+  }
+  return true;
+}
+#define B2A_DBG(cond) (!::b2a::kDebugBuild || ::b2a::dbg_check(cond))
+
+__device__ __forceinline__ int warp_quarter() { return static_cast<int>((threadIdx.x >> 5) & 3u); }
+
+__device__ __forceinline__ uint32_t dyn_smem_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(r));
+  return r;
+}
 
 // Wall-clock limit of one bounded wait.  A healthy wait in these kernels is
 // microseconds; two seconds means a lost arrival.
@@ -241,6 +276,7 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 // D[tmem] (+)= A[smem desc] * B[smem desc]; kind::f16, fp32 accumulate.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
+  if (!B2A_DBG(tmem_operand_ok(d_tmem, idesc_n(idesc)))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -252,6 +288,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
 // D[tmem] (+)= A[tmem] * B[smem desc]; A is K-major fp16 packed two per column.
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
+  if (!B2A_DBG(tmem_operand_ok(d_tmem, idesc_n(idesc)) && tmem_operand_ok(a_tmem, 8))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -295,6 +332,11 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn_maj
                   "r"(r[b + 4]), "r"(r[b + 5]), "r"(r[b + 6]), "r"(r[b + 7])
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  if (!B2A_DBG(tmem_ldst_ok(taddr, 32, warp_quarter()))) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = 0u;
+    return;
+  }
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -304,6 +346,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  if (!B2A_DBG(tmem_ldst_ok(taddr, 32, warp_quarter()))) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
@@ -314,6 +357,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  if (!B2A_DBG(tmem_ldst_ok(taddr, 16, warp_quarter()))) return;
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
@@ -390,6 +434,7 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 
 __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
+  if (!B2A_DBG(tmem_operand_ok(d_tmem, idesc_n(idesc)))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -400,6 +445,7 @@ __device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t adesc, uin
 
 __device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                             uint32_t idesc, uint32_t accumulate) {
+  if (!B2A_DBG(tmem_operand_ok(d_tmem, idesc_n(idesc)) && tmem_operand_ok(a_tmem, 8))) return;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
@@ -438,6 +484,37 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
       : "memory");
+}
+
+// ----------------------------------------------- checked TMA tile loads ----
+// The loads above with the debug build's checks: the box start (x, y, z)
+// against the map's innermost extent nx (fp16 elements), y against ny and z
+// against the end nz of the rows the launch covers; the destination's
+// ``bytes`` against the CTA's dynamic shared memory starting at
+// ``smem_base``.  A failed check skips the copy (its barrier then never
+// completes, and the waits give up at once on the set status word).
+
+__device__ __forceinline__ bool tma_box_checked(uint32_t dst, uint32_t bytes, uint32_t smem_base, int x, int nx,
+                                                int y, int ny, int z, int nz) {
+  return B2A_DBG(tma_coords_ok(x, 2, nx, y, ny, z, nz) && smem_box_ok(dst, bytes, smem_base, dyn_smem_size()));
+}
+
+__device__ __forceinline__ void tma_load_3d_chk(uint32_t dst, uint32_t bytes, uint32_t smem_base,
+                                                const CUtensorMap* map, uint32_t bar, int x, int y, int z, int nx,
+                                                int ny, int nz) {
+  if (tma_box_checked(dst, bytes, smem_base, x, nx, y, ny, z, nz)) tma_load_3d(dst, map, bar, x, y, z);
+}
+
+__device__ __forceinline__ void tma_load_3d_pair_chk(uint32_t dst, uint32_t bytes, uint32_t smem_base,
+                                                     const CUtensorMap* map, uint32_t leader_bar, int x, int y,
+                                                     int z, int nx, int ny, int nz) {
+  if (tma_box_checked(dst, bytes, smem_base, x, nx, y, ny, z, nz)) tma_load_3d_pair(dst, map, leader_bar, x, y, z);
+}
+
+__device__ __forceinline__ void tma_load_2d_pair_chk(uint32_t dst, uint32_t bytes, uint32_t smem_base,
+                                                     const CUtensorMap* map, uint32_t leader_bar, int x, int z,
+                                                     int nx, int nz) {
+  if (tma_box_checked(dst, bytes, smem_base, x, nx, 0, 1, z, nz)) tma_load_2d_pair(dst, map, leader_bar, x, z);
 }
 
 // ------------------------------------------------------------ arithmetic ----

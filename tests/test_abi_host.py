@@ -31,11 +31,22 @@ def test_every_declared_symbol_is_exported(lib):
         assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
 
 
+def test_debug_build_exports_the_same_entry_points():
+    path = B.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    dbg.b2a_debug_build.restype = ctypes.c_int
+    assert dbg.b2a_debug_build() == 1
+
+
 def test_version_and_status_strings(lib):
-    assert lib.b2a_version() == 103
+    assert lib.b2a_version() == 104
+    assert lib.b2a_debug_build() == 0
     assert lib.b2a_status_string(0) == b"ok"
     assert lib.b2a_status_string(1) == b"invalid argument"
     assert lib.b2a_status_string(4) == b"device-side wait timed out"
+    assert lib.b2a_status_string(5) == b"device-side bounds check failed (debug build)"
     assert lib.b2a_status_string(99) == b"unknown status"
 
 

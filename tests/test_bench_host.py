@@ -67,3 +67,9 @@ class _FakeLib:
 ])
 def test_kernel_names_match_the_launch_list(choice, mode, name):
     assert bench.attn_kernel_name(_FakeLib(choice), 128, 4096, mode) == name
+
+
+def test_merge_kernel_names():
+    assert bench.merge_kernel_name(128, 8, "float") == "attn_merge_pipe_kernel<128, float>"
+    assert bench.merge_kernel_name(128, 16, "float") == "attn_merge_pipe_kernel<128, float>"
+    assert bench.merge_kernel_name(64, 17, "float") == "attn_merge_kernel<64, float>"
