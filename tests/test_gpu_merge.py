@@ -46,3 +46,22 @@ def test_merge_full_size_sampled(b2a):
     ref, ref_lse = OC.merge(o[:, rows], lse[:, :, rows])
     assert_out_close(out.cpu().numpy()[rows].astype(np.float64), ref, "merge 32k sampled")
     assert_lse_close(lse_out.cpu().numpy()[:, rows], ref_lse)
+
+
+@pytest.mark.parametrize("P,dtype", [(5, "f32"), (9, "f32"), (9, "f16")])
+def test_merge_many_pair_groups_per_block(b2a, P, dtype):
+    # 155400 (row, head) pairs = 607 groups of 256, the last one partial (8
+    # pairs): every block of the persistent merge (two per SM) walks two or
+    # three groups with its weights double-buffered across them, and P = 9
+    # streams its chunks in two batches; all pairs against the oracle
+    S, H, d = 4200, 37, 64
+    o, lse = W.merge_operands(P, S, H, d, seed=P + 77, empty_chunks=(1,))
+    if dtype == "f16":
+        o = o.astype(np.float16)
+        out, lse_out = b2a.attn_merge_f16(torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda())
+    else:
+        out, lse_out = b2a.attn_merge(torch.from_numpy(o).cuda(), torch.from_numpy(lse).cuda())
+    b2a.check_status()
+    ref, ref_lse = OC.merge(o, lse)
+    assert_out_close(out.cpu().numpy().astype(np.float64), ref, f"merge {dtype} P={P}, 607 pair groups")
+    assert_lse_close(lse_out.cpu().numpy(), ref_lse)
