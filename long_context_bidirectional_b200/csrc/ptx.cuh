@@ -20,7 +20,9 @@ enum : uint32_t {
 };
 
 // The library's device status word (one per device, static device memory):
-// set by kernels, read and cleared by b2a_check_status().
+// set by kernels, read and cleared by b2a_check_status().  Defined here
+// because the whole library is one translation unit (b200attn.cu includes
+// every kernel header), so device code anywhere in it can name the word.
 __device__ unsigned int g_status_word;
 
 #ifdef B2A_DEBUG
