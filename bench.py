@@ -773,7 +773,10 @@ def run_reference(args, rank, world):
                           "workloads only"}), flush=True)
         return
     w = W.ATTN_WORKLOADS[args.workload]
-    rows = 8  # query rows per head per step: a bounded sample of the workload
+    # query rows per head per step: a bounded sample of the workload, large
+    # enough that the oracle's arithmetic (not its per-call widening of K and
+    # V to FP64) dominates a step (~1-2 s on 16 host cores)
+    rows = 32
     for _ in range(args.warmup):
         oracle_sample(w, rows)
     total_flops, total_s = 0.0, 0.0
